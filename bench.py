@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the Ca2-VDM cached attention path on B200.
+
+One step = one autoregressive step at steady state of the Open-Sora-v1.0-shaped attention
+layer with the full Pmax = 41 queue (B=1, 256 tokens/frame, 16 heads x 72, chunk l = 8,
+P' = 3, T = 50 denoising steps): for each of the 28 blocks of the backbone (each with its
+own cache, as in the model), T denoising passes of prefix-spatial + causal temporal
+attention reading the shared cache, then the cache-writing pass (self-repeat spatial +
+temporal), eviction of the 8 oldest frames, the cache write for all blocks, and the
+chunk's cyclic TPE indices.  28 per-block caches plus their inputs (~2.4 GB) keep every
+read coming from HBM (inputs larger than L2).
+
+Metric: attention query tokens per second -- each pass moves B*l*HW = 2048 query tokens
+through one block's spatial + temporal attention, so a step counts (T+1) * 28 * 2048.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun each rank runs the same step on its own GPU with its own caches (videos
+are independent; no data-path collective); value = all ranks' tokens / max rank time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn query-tokens/s per denoise step; temporal HBM GB/s; spatial TFLOP/s vs peak"
+WORKLOAD = dict(batch=1, hw=256, heads=16, head_dim=72, chunk_len=8, p_max=41, p_spatial=3,
+                n_layers=28, denoise_steps=50)
+WORKLOAD_NAME = ("Open-Sora-shaped attention layer, Pmax=41 full queue (steady-state AR step of the "
+                 "80-frame run), 28 per-block caches")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ca2", choices=["ca2", "reference"])
+    ap.add_argument("--layers", type=int, default=WORKLOAD["n_layers"])
+    ap.add_argument("--denoise", type=int, default=WORKLOAD["denoise_steps"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ------------------------------------------------------------------------------------
+class Clocks:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def source_sha(name: str) -> str:
+    with open(os.path.join(ROOT, "causal_kv_cache_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel_file: str):
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            d = json.load(f)
+        e = d.get(kernel_file)
+        if e and e.get("source_sha") == source_sha(kernel_file):
+            return e.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------------
+def run_ca2(args):
+    import torch
+    import torch.distributed as dist
+    from causal_kv_cache_b200 import ca2
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    W = dict(WORKLOAD, n_layers=args.layers, denoise_steps=args.denoise)
+    B, HW, H, D, l, PM, PS = (W[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max", "p_spatial"))
+    NL, T = W["n_layers"], W["denoise_steps"]
+    plane = B * HW * H * D
+    frame_bytes = plane * 2
+    cache = ca2.KVCache(NL, B, HW, H, D, l, PM, PS)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + rank)
+
+    def rnd(n):
+        return (torch.randn((B, n, HW, H, D), generator=g, device=dev) * 0.7).to(torch.bfloat16)
+
+    # per-block inputs (queries/keys/values for both attentions), reused across passes
+    inp = [dict(sq=rnd(l), sk=rnd(l), sv=rnd(l), tq=rnd(l), tk=rnd(l), tv=rnd(l)) for _ in range(NL)]
+    so = [torch.empty((B, l, HW, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    to = [torch.empty((B, l, HW, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+
+    # fill the queue: first frame + 5 chunks -> 41 frames, spatial cache 3
+    for n in (1, 8, 8, 8, 8, 8):
+        ks = [rnd(n) for _ in range(NL)]
+        vs = [rnd(n) for _ in range(NL)]
+        cache.evict_for(n)
+        cache.write(ks, vs, ks, vs, n, sp)
+    torch.cuda.synchronize()
+    assert cache.state()[1] == PM
+
+    h = cache.handle
+    tempo = ca2.ca2_temporal_attn
+    spat = ca2.ca2_spatial_prefix_attn
+    ptr = lambda t: t.data_ptr()
+    P = [{k: ptr(v) for k, v in d.items()} for d in inp]
+    SO = [ptr(t) for t in so]
+    TO = [ptr(t) for t in to]
+    KT = [P[L]["tk"] for L in range(NL)]
+    VT = [P[L]["tv"] for L in range(NL)]
+    KS = [P[L]["sk"] for L in range(NL)]
+    VS = [P[L]["sv"] for L in range(NL)]
+    g0 = [1 + 8 * 5]
+
+    timed_passes = {0, T // 2, T}      # passes whose launches carry CUDA events
+
+    def step(ev=None):
+        """One AR step.  ev: optional list collecting per-launch event pairs."""
+        ca2.ca2_tpe_indices(h, g0[0], 0, l)
+        for t in range(T + 1):
+            use_prefix = 1 if t < T else 0
+            rec = ev is not None and t in timed_passes
+            for L in range(NL):
+                p = P[L]
+                if rec:
+                    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                    e0.record(stream)
+                spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, sp)
+                if rec:
+                    e1.record(stream)
+                tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, sp)
+                if rec:
+                    e2.record(stream)
+                    ev.append(("den" if use_prefix else "self", e0, e1, e2))
+        cache.evict_for(l)
+        if ev is not None:
+            e3, e4 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            e3.record(stream)
+        ca2.ca2_cache_write(h, KT, VT, KS, VS, l, sp)
+        if ev is not None:
+            e4.record(stream)
+            ev.append(("write", e3, e4, None))
+        g0[0] += l
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ca2.ca2_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after warm-up" % st)
+
+    clocks = Clocks(local)
+    ev = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(ev)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    st = ca2.ca2_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after the timed region" % st)
+
+    sp_den, sp_self, tp_ms, wr_ms = [], [], [], []
+    for kind, a, b_, c in ev:
+        if kind == "write":
+            wr_ms.append(a.elapsed_time(b_))
+            continue
+        (sp_den if kind == "den" else sp_self).append(a.elapsed_time(b_))
+        tp_ms.append(b_.elapsed_time(c))
+    resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * plane) * 2 / 1e9
+    launches_per_step = (T + 1) * NL * 2 + 1
+    tokens_per_step = (T + 1) * NL * B * l * HW
+    value = tokens_per_step * args.steps * world / (ms / 1e3)
+
+    # ---- roofline of each kernel ----
+    pk, pk_kind = peaks()
+    t_bytes = (2 * PM + 4 * l) * frame_bytes                       # cache K,V + chunk Q,K,V + O
+    s_flops_den = 4 * D * HW * (1 + PS) * HW * l * H * B           # denoising mode (P' prefix frames)
+    s_flops_self = 4 * D * HW * HW * l * H * B                     # self-repeat mode (own frame once)
+    w_bytes = 2 * NL * (2 * l + 2 * PS) * frame_bytes              # read + write of K,V (temporal, spatial)
+    avg_t = statistics.mean(tp_ms) / 1e3
+    avg_sd = statistics.mean(sp_den) / 1e3
+    avg_ss = statistics.mean(sp_self) / 1e3
+    avg_w = statistics.mean(wr_ms) / 1e3
+    kernels = {
+        "temporal": {"bound": "hbm", "us": avg_t * 1e6, "achieved": t_bytes / avg_t / 1e9,
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": t_bytes},
+        "spatial": {"bound": "tensor", "us": avg_sd * 1e6, "achieved": s_flops_den / avg_sd / 1e12,
+                    "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "flops_per_launch": s_flops_den},
+        "spatial_self": {"bound": "tensor", "us": avg_ss * 1e6, "achieved": s_flops_self / avg_ss / 1e12,
+                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "flops_per_launch": s_flops_self},
+        "cache_write": {"bound": "hbm", "us": avg_w * 1e6, "achieved": w_bytes / avg_w / 1e9,
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": w_bytes},
+    }
+    for k in kernels.values():
+        k["frac"] = k["achieved"] / k["peak"]
+    step_s = ms / 1e3 / args.steps
+    share_t = avg_t * (T + 1) * NL / step_s
+    share_s = (avg_sd * T + avg_ss) * NL / step_s
+    share_w = avg_w / step_s
+    dom = "temporal" if share_t >= share_s else "spatial"
+    dk = kernels[dom]
+    traffic = committed_traffic("k_temporal.cu" if dom == "temporal" else "k_spatial.cu")
+    roofline = {"kernel": "k_temporal_causal" if dom == "temporal" else "k_spatial_prefix",
+                "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
+                "frac": dk["frac"], "traffic": traffic, "peak_source": pk_kind}
+
+    # ---- end to end through host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cache, inp, so, to, step, stream, NL, tokens_per_step, world, dist)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.49) bf16 Q/K/V; no weights needed)",
+        "config": {"workload": WORKLOAD_NAME, "batch": B, "tokens_per_frame": HW, "heads": H,
+                   "head_dim": D, "chunk_len": l, "p_max": PM, "p_spatial": PS, "blocks": NL,
+                   "denoise_steps": T, "queue_len": PM, "parallelism": "replica per GPU (dp%d)" % world,
+                   "l2": "inputs larger than L2: %d per-block caches and inputs, %.2f GB on the device"
+                         % (NL, resident_gb),
+                   "tokens_per_step": tokens_per_step},
+        "roofline": roofline,
+        "kernels": kernels,
+        "kernel_time_share": {"temporal": share_t, "spatial": share_s, "cache_write": share_w},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=12.0)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def run_e2e(args, cache, inp, so, to, step_fn, stream, NL, tokens_per_step, world, dist):
+    """The same step with its inputs copied from pinned host memory and its outputs read
+    back, all inside the timed region."""
+    import torch
+    host_in = [{k: v.cpu().pin_memory() for k, v in d.items()} for d in inp]
+    host_out = [torch.empty(so[0].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2 * NL)]
+    h2d = sum(v.numel() * 2 for d in host_in for v in d.values())
+    d2h = sum(t.numel() * 2 for t in host_out)
+
+    def e2e_step():
+        for L in range(NL):
+            for k, v in host_in[L].items():
+                inp[L][k].copy_(v, non_blocking=True)
+        step_fn()
+        for L in range(NL):
+            host_out[2 * L].copy_(so[L], non_blocking=True)
+            host_out[2 * L + 1].copy_(to[L], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 5))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    return {"value": tokens_per_step * steps * world / (ms / 1e3), "unit": "query-tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ------------------------------------------------------------------------------------
+def oracle_sample(budget_s: float):
+    """Time the fp64 oracle on a bounded sample of one block's pass (all host threads).
+
+    Sample: temporal attention for 64 token positions x 16 heads (8 queries, 41 queued +
+    8 chunk keys each) and prefix-spatial attention for 2 frame-heads (256 queries x 1024
+    keys), scaled to query tokens of one block pass (all heads)."""
+    import numpy as np
+    import oracle
+    from ca2_synth import Generator, WORKLOADS
+    wl = WORKLOADS["os_p41"]
+    gen = Generator(wl, 0)
+    q, k, v = gen.qkv(wl.chunk_len)
+    _, pk, pv = gen.qkv(wl.p_max)
+    prefix_k = [pk[:, i] for i in range(wl.p_max)]
+    prefix_v = [pv[:, i] for i in range(wl.p_max)]
+    sk = prefix_k[-3:]
+    sv = prefix_v[-3:]
+    H = wl.heads
+    t_units = np.arange(64 * H)
+    s_units = np.arange(2)
+    t_time = s_time = 0.0
+    reps = 0
+    start = time.perf_counter()
+    while True:
+        a = time.perf_counter()
+        oracle.temporal_attn(q, k, v, prefix_k, prefix_v, units=t_units)
+        b = time.perf_counter()
+        oracle.spatial_attn(q, k, v, sk, sv, repeat=0, units=s_units)
+        c = time.perf_counter()
+        t_time += b - a
+        s_time += c - b
+        reps += 1
+        if time.perf_counter() - start > budget_s:
+            break
+    # seconds per query token (all heads): temporal sample = 64 positions x 8 frames,
+    # spatial sample = 2/16 of one frame's 256 query tokens
+    t_per_tok = (t_time / reps) / (64 * wl.chunk_len)
+    s_per_tok = (s_time / reps) / (256 * len(s_units) / H)
+    value = 1.0 / (t_per_tok + s_per_tok)
+    sample = ("%d reps of: temporal 64 positions x 16 heads x 8 queries over 49 keys; spatial 2 "
+              "frame-heads x 256 queries x 1024 keys (Pmax=41, P'=3 shapes); scaled to query tokens "
+              "of one block pass" % reps)
+    return value, sample, oracle.num_threads(), time.perf_counter() - start
+
+
+def cpu_baseline(budget_s: float):
+    value, sample, cores, _ = oracle_sample(budget_s)
+    return {"value": value, "unit": "query-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle_sample(budget_s=0.5)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, sample, cores, _ = oracle_sample(budget_s=3.0)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD_NAME, "sample": "bounded CPU sample per step"},
+        "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ca2(args)
+
+
+if __name__ == "__main__":
+    main()

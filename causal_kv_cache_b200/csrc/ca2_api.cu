@@ -1,0 +1,344 @@
+// ca2_api.cu -- the extern "C" surface of libca2.so (declared in include/ca2.h).
+//
+// Host side of the Ca2-VDM cached attention path: argument validation, the ring-buffer
+// state of the temporal KV-cache queue (head / count kept on the host and passed to the
+// kernels by value), the spatial-cache frame count, cyclic TPE indices, tensor-map
+// encoding for the tensor-core kernel, and kernel launches on the caller's stream.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ca2.h"
+#include "ca2_kernels.h"
+
+struct ca2_cache {
+    ca2_config cfg;
+    uint8_t *tbuf;      // [N_L][2][Pmax][B][HW][H][D] bf16
+    uint8_t *sbuf;      // [N_L][2][P'][B][HW][H][D] bf16
+    size_t plane_bytes; // bytes of one frame-plane B*HW*H*D*2
+    int head;           // ring slot of the oldest queued frame
+    int count;          // queued frames
+    int sp_count;       // frames in the spatial cache
+    long long frames_written;
+};
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_config(const ca2_config *c)
+{
+    if (!c) return CA2_ERR_ARG;
+    if (c->n_layers < 1 || c->batch < 1 || c->hw < 1 || c->heads < 1) return CA2_ERR_SHAPE;
+    if (c->head_dim < 8 || c->head_dim > 128 || (c->head_dim % 8) != 0) return CA2_ERR_SHAPE;
+    if (c->chunk_len < 1 || c->chunk_len > ca2::kMaxChunk) return CA2_ERR_SHAPE;
+    if (c->p_max < c->chunk_len) return CA2_ERR_SHAPE;
+    if (c->p_spatial < 0 || c->p_spatial > c->chunk_len) return CA2_ERR_SHAPE;
+    if (c->tpe_len < 0) return CA2_ERR_SHAPE;
+    // tensor-map extents and 32-bit strides
+    const long long hd = (long long)c->heads * c->head_dim;
+    if (hd * c->hw * 2 > (1ll << 40) || c->hw > (1 << 30)) return CA2_ERR_SHAPE;
+    return CA2_OK;
+}
+
+size_t plane_bytes_of(const ca2_config *c)
+{
+    return (size_t)c->batch * (size_t)c->hw * (size_t)c->heads * (size_t)c->head_dim * 2u;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CA2_OK : CA2_ERR_CUDA; }
+
+int sm_count()
+{
+    static int cached_dev = -1, cached = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev != cached_dev) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached = n;
+        cached_dev = dev;
+    }
+    return cached;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// View a bf16 tensor [frames][HW][H][D] as 4-D (D, H, HW, frames) and encode a tiled map.
+bool encode_4d(CUtensorMap *m, const void *base, int D, int H, int HW, int frames, int box_d, int box_rows,
+               CUtensorMapSwizzle swz)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)HW, (cuuint64_t)frames};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)HW * H * D * 2};
+    cuuint32_t box[4] = {(cuuint32_t)box_d, 1u, (cuuint32_t)box_rows, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+uint8_t *layer_ring(const ca2_cache *c, int layer, int kv)
+{
+    return c->tbuf + ((size_t)layer * 2 + (size_t)kv) * (size_t)c->cfg.p_max * c->plane_bytes;
+}
+
+uint8_t *layer_spatial(const ca2_cache *c, int layer, int kv)
+{
+    return c->sbuf + ((size_t)layer * 2 + (size_t)kv) * (size_t)c->cfg.p_spatial * c->plane_bytes;
+}
+
+int check_chunk_args(const ca2_cache *c, int layer, const void *q, const void *k, const void *v, const void *out,
+                     int n)
+{
+    if (!c || !q || !k || !v || !out) return CA2_ERR_ARG;
+    if (layer < 0 || layer >= c->cfg.n_layers) return CA2_ERR_ARG;
+    if (n < 1 || n > c->cfg.chunk_len) return CA2_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return CA2_ERR_ALIGN;
+    return CA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ca2_cache_bytes(const ca2_config *cfg, size_t *temporal_bytes, size_t *spatial_bytes)
+{
+    int st = validate_config(cfg);
+    if (st != CA2_OK) return st;
+    const size_t plane = plane_bytes_of(cfg);
+    if (temporal_bytes) *temporal_bytes = 2u * (size_t)cfg->n_layers * (size_t)cfg->p_max * plane;
+    if (spatial_bytes) *spatial_bytes = 2u * (size_t)cfg->n_layers * (size_t)cfg->p_spatial * plane;
+    return CA2_OK;
+}
+
+int ca2_cache_init(const ca2_config *cfg, void *temporal_buf, size_t temporal_bytes, void *spatial_buf,
+                   size_t spatial_bytes, ca2_cache **out)
+{
+    if (!out) return CA2_ERR_ARG;
+    *out = nullptr;
+    int st = validate_config(cfg);
+    if (st != CA2_OK) return st;
+    size_t need_t = 0, need_s = 0;
+    ca2_cache_bytes(cfg, &need_t, &need_s);
+    if (!temporal_buf) return CA2_ERR_ARG;
+    if (need_s > 0 && !spatial_buf) return CA2_ERR_ARG;
+    if (temporal_bytes < need_t || spatial_bytes < need_s) return CA2_ERR_CAPACITY;
+    if (!aligned16(temporal_buf) || (spatial_buf && !aligned16(spatial_buf))) return CA2_ERR_ALIGN;
+    ca2_cache *c = new (std::nothrow) ca2_cache;
+    if (!c) return CA2_ERR_ARG;
+    c->cfg = *cfg;
+    if (c->cfg.tpe_len == 0) c->cfg.tpe_len = cfg->p_max + cfg->chunk_len;
+    c->tbuf = static_cast<uint8_t *>(temporal_buf);
+    c->sbuf = static_cast<uint8_t *>(spatial_buf);
+    c->plane_bytes = plane_bytes_of(cfg);
+    c->head = 0;
+    c->count = 0;
+    c->sp_count = 0;
+    c->frames_written = 0;
+    *out = c;
+    return CA2_OK;
+}
+
+int ca2_cache_destroy(ca2_cache *cache)
+{
+    delete cache;
+    return CA2_OK;
+}
+
+int ca2_cache_evict(ca2_cache *c, int n)
+{
+    if (!c) return CA2_ERR_ARG;
+    if (n < 0 || n > c->count) return CA2_ERR_CAPACITY;
+    c->head = (c->head + n) % c->cfg.p_max;
+    c->count -= n;
+    return CA2_OK;
+}
+
+int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t, const void *const *k_s,
+                    const void *const *v_s, int n, void *stream)
+{
+    if (!c || !k_t || !v_t) return CA2_ERR_ARG;
+    const ca2_config &g = c->cfg;
+    if (n < 1 || n > g.chunk_len) return CA2_ERR_SHAPE;
+    if (c->count + n > g.p_max) return CA2_ERR_CAPACITY;
+    const int n_sp = n < g.p_spatial ? n : g.p_spatial;
+    if (n_sp > 0 && (!k_s || !v_s)) return CA2_ERR_ARG;
+    for (int L = 0; L < g.n_layers; ++L) {
+        if (!k_t[L] || !v_t[L]) return CA2_ERR_ARG;
+        if (!aligned16(k_t[L]) || !aligned16(v_t[L])) return CA2_ERR_ALIGN;
+        if (n_sp > 0) {
+            if (!k_s[L] || !v_s[L]) return CA2_ERR_ARG;
+            if (!aligned16(k_s[L]) || !aligned16(v_s[L])) return CA2_ERR_ALIGN;
+        }
+    }
+    ca2::CacheWriteParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.tbuf = reinterpret_cast<uint4 *>(c->tbuf);
+    p.sbuf = reinterpret_cast<uint4 *>(c->sbuf);
+    p.plane_vec = (long long)(c->plane_bytes / (size_t)g.batch / 16u);
+    p.n = n;
+    p.B = g.batch;
+    p.slot0 = (c->head + c->count) % g.p_max;
+    p.p_max = g.p_max;
+    p.n_sp = n_sp;
+    p.p_spatial = g.p_spatial;
+    for (int L0 = 0; L0 < g.n_layers; L0 += ca2::kMaxLayersPerWrite) {
+        const int nl = (g.n_layers - L0) < ca2::kMaxLayersPerWrite ? (g.n_layers - L0) : ca2::kMaxLayersPerWrite;
+        p.layer0 = L0;
+        p.n_layers = nl;
+        for (int i = 0; i < nl; ++i) {
+            p.layer[i].kt = static_cast<const uint4 *>(k_t[L0 + i]);
+            p.layer[i].vt = static_cast<const uint4 *>(v_t[L0 + i]);
+            p.layer[i].ks = n_sp > 0 ? static_cast<const uint4 *>(k_s[L0 + i]) : nullptr;
+            p.layer[i].vs = n_sp > 0 ? static_cast<const uint4 *>(v_s[L0 + i]) : nullptr;
+        }
+        cudaError_t e = ca2::launch_cache_write(p, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return CA2_ERR_CUDA;
+    }
+    c->count += n;
+    c->sp_count = n_sp;
+    c->frames_written += n;
+    return CA2_OK;
+}
+
+int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, const void *v, void *out, int n,
+                      void *stream)
+{
+    int st = check_chunk_args(c, layer, q, k, v, out, n);
+    if (st != CA2_OK) return st;
+    const ca2_config &g = c->cfg;
+    ca2::TemporalParams p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.ring_k = reinterpret_cast<const __nv_bfloat16 *>(layer_ring(c, layer, 0));
+    p.ring_v = reinterpret_cast<const __nv_bfloat16 *>(layer_ring(c, layer, 1));
+    p.B = g.batch;
+    p.HW = g.hw;
+    p.H = g.heads;
+    p.D = g.head_dim;
+    p.n = n;
+    p.Pk = c->count;
+    p.head = c->head;
+    p.Pmax = g.p_max;
+    int G = ca2::kMaxTemporalGroup;
+    while (g.heads % G) G >>= 1;
+    p.G = G;
+    p.n_items = g.batch * g.hw * (g.heads / G);
+    p.n_stages = (c->count + n + 15) / 16;
+    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
+    p.row_bytes = (uint32_t)(G * g.head_dim * 2);
+    p.pitch = ca2::temporal_pitch(G, g.head_dim);
+    const int sms = sm_count();
+    if (sms <= 0) return CA2_ERR_CUDA;
+    int grid = 2 * sms;
+    if (grid > p.n_items) grid = p.n_items;
+    return cuda_status(ca2::launch_temporal(p, grid, static_cast<cudaStream_t>(stream)));
+}
+
+int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *k, const void *v, void *out,
+                            int n, int use_prefix, void *stream)
+{
+    int st = check_chunk_args(c, layer, q, k, v, out, n);
+    if (st != CA2_OK) return st;
+    if (use_prefix != 0 && use_prefix != 1) return CA2_ERR_ARG;
+    const ca2_config &g = c->cfg;
+    const int n_sp = use_prefix ? c->sp_count : 0;
+    const int frames = g.batch * n;
+    ca2::SpatialMaps m;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_32B;
+    bool ok = encode_4d(&m.q, q, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
+              encode_4d(&m.k, k, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
+              encode_4d(&m.v, v, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
+              encode_4d(&m.o, out, g.head_dim, g.heads, g.hw, frames, g.head_dim, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && n_sp > 0) {
+        ok = encode_4d(&m.sk, layer_spatial(c, layer, 0), g.head_dim, g.heads, g.hw, n_sp * g.batch, 16, 128, sw) &&
+             encode_4d(&m.sv, layer_spatial(c, layer, 1), g.head_dim, g.heads, g.hw, n_sp * g.batch, 16, 128, sw);
+    } else if (ok) {
+        m.sk = m.k;   // never read when there is no prefix
+        m.sv = m.v;
+    }
+    if (!ok) return CA2_ERR_CUDA;
+    ca2::SpatialParams p;
+    p.B = g.batch;
+    p.n = n;
+    p.H = g.heads;
+    p.HW = g.hw;
+    p.D = g.head_dim;
+    p.n_src = 1 + n_sp;
+    p.nkb = (g.hw + 127) / 128;
+    p.q_tiles = (g.hw + 127) / 128;
+    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
+    return cuda_status(ca2::launch_spatial(m, p, static_cast<cudaStream_t>(stream)));
+}
+
+int ca2_tpe_indices(const ca2_cache *c, long long first_global_frame, int offset, int n, int *out_host)
+{
+    if (!c) return CA2_ERR_ARG;
+    if (n < 0 || first_global_frame < 0 || offset < 0) return CA2_ERR_ARG;
+    if (n > 0 && !out_host) return CA2_ERR_ARG;
+    const long long N = c->cfg.tpe_len;
+    for (int i = 0; i < n; ++i) out_host[i] = (int)(((long long)offset + first_global_frame + i) % N);
+    return CA2_OK;
+}
+
+int ca2_cache_state(const ca2_cache *c, int *head, int *count, int *sp_count, long long *frames_written)
+{
+    if (!c) return CA2_ERR_ARG;
+    if (head) *head = c->head;
+    if (count) *count = c->count;
+    if (sp_count) *sp_count = c->sp_count;
+    if (frames_written) *frames_written = c->frames_written;
+    return CA2_OK;
+}
+
+int ca2_device_status(void)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) return CA2_ERR_CUDA;
+    int s = 0;
+    if (ca2::read_and_clear_status(&s) != 0) return CA2_ERR_CUDA;
+    return s == 0 ? CA2_OK : CA2_ERR_TIMEOUT;
+}
+
+int ca2_selftest_timeout(int wait_us, void *stream)
+{
+    if (wait_us < 1 || wait_us > 1000000) return CA2_ERR_ARG;
+    return cuda_status(
+        ca2::launch_timeout_selftest((unsigned long long)wait_us * 1000ull, static_cast<cudaStream_t>(stream)));
+}
+
+const char *ca2_status_string(int s)
+{
+    switch (s) {
+    case CA2_OK: return "ok";
+    case CA2_ERR_ARG: return "invalid argument";
+    case CA2_ERR_SHAPE: return "size outside the supported range";
+    case CA2_ERR_CAPACITY: return "capacity exceeded";
+    case CA2_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case CA2_ERR_CUDA: return "CUDA runtime error";
+    case CA2_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+/*
+ * ca2.h -- C ABI of libca2.so: the Ca2-VDM cached attention path on one NVIDIA B200.
+ *
+ * Ca2-VDM (arXiv 2411.16375, "Ca2-VDM: Efficient Autoregressive Video Diffusion Model with
+ * Causal Generation and Cache Sharing"; ICML 2025 papernotes page, sections 整体框架 and
+ * 关键设计 1-5) generates video chunk by chunk.  Each autoregressive (AR) step runs T
+ * denoising steps that READ a KV cache of clean prefix frames, then one cache-writing
+ * pass over the denoised chunk that APPENDS its K/V.  The cache does not depend on the
+ * denoising step (prefix frames use tEmb(0)), so one copy serves all T steps.
+ *
+ * Conventions shared by every call:
+ *   - Elements are bfloat16.  Chunk tensors (q, k, v, out) are dense, row-major
+ *     [B][n][HW][H][D]: video, frame of the chunk, spatial token, head, head dim.
+ *     All device pointers must be 16-byte aligned.
+ *   - The caller owns all device memory (allocate it however you like, e.g. torch).
+ *     The library stores the two cache pointers given to ca2_cache_init and never
+ *     frees or reallocates them.
+ *   - Device calls are asynchronous on the caller's stream (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream) and never synchronise.  Ring indices live
+ *     on the host and reach the kernels as launch arguments, so host state advances at
+ *     call time: issue calls in the order they must execute.
+ *   - Errors are returned as ca2_status codes.  Nothing aborts, throws or traps.  A
+ *     launch failure is CA2_ERR_CUDA.  A kernel whose bounded wait gave up records it in a
+ *     device status word, read (with a device synchronisation) by ca2_device_status.
+ *   - A handle is not thread-safe.
+ *
+ * Cache memory layout (both buffers caller-allocated, sizes from ca2_cache_bytes):
+ *   temporal: [N_L][2][Pmax][B][HW][H][D]   (index 0 = K ring, 1 = V ring)
+ *   spatial : [N_L][2][P'][B][HW][H][D]
+ * A ring slot is one frame-plane [B][HW][H][D] with exactly the layout of one frame of
+ * a chunk tensor.  The i-th oldest queued frame (i = 0 .. count-1) is in slot
+ * (head + i) mod Pmax; spatial slot j (j < sp_count) holds the j-th of the last
+ * sp_count frames written, oldest first.
+ *
+ * Required order within one AR step:
+ *   T x { for each layer: ca2_spatial_prefix_attn(use_prefix=1), ca2_temporal_attn }
+ *   cache-writing pass: for each layer: ca2_spatial_prefix_attn(use_prefix=0), ca2_temporal_attn
+ *   ca2_cache_evict(max(0, count + n - Pmax))   then   ca2_cache_write(n)
+ * The pass's attention reads the queue before eviction overwrites its oldest slots;
+ * stream order keeps that true on the device.
+ */
+#ifndef CA2_H
+#define CA2_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ca2_cache ca2_cache;   /* opaque host-side handle */
+
+typedef struct {
+    int n_layers;   /* N_L >= 1: attention blocks, each with its own cache                */
+    int batch;      /* B >= 1 videos                                                       */
+    int hw;         /* HW >= 1 spatial tokens per frame                                    */
+    int heads;      /* H >= 1                                                              */
+    int head_dim;   /* D: multiple of 8, 8 <= D <= 128                                     */
+    int chunk_len;  /* l: frames per AR chunk, 1 <= l <= 8                                 */
+    int p_max;      /* Pmax >= l: capacity of the temporal queue, in frames                */
+    int p_spatial;  /* P': 0 <= P' <= l prefix frames kept for spatial attention           */
+    int tpe_len;    /* N_tpe >= 1: temporal positional table length; 0 selects Pmax + l     */
+} ca2_config;
+
+typedef enum {
+    CA2_OK = 0,
+    CA2_ERR_ARG = -1,       /* null pointer, bad flag, layer out of range                 */
+    CA2_ERR_SHAPE = -2,     /* a size outside the documented range                        */
+    CA2_ERR_CAPACITY = -3,  /* write would overflow the queue, or a buffer is too small   */
+    CA2_ERR_ALIGN = -4,     /* a pointer is not 16-byte aligned                           */
+    CA2_ERR_CUDA = -5,      /* a CUDA runtime call or kernel launch failed                */
+    CA2_ERR_TIMEOUT = -6    /* a kernel's bounded wait gave up (see ca2_device_status)     */
+} ca2_status;
+
+/* Sizes in bytes of the temporal and spatial cache buffers for a configuration:
+ * temporal = 2 * N_L * Pmax * B*HW*H*D * 2, spatial = 2 * N_L * P' * B*HW*H*D * 2.
+ * One cache serves every denoising step (papernotes page, 关键设计 2), so the size has
+ * no factor T.  Either out pointer may be NULL.  CA2_ERR_SHAPE on an invalid config. */
+int ca2_cache_bytes(const ca2_config *cfg, size_t *temporal_bytes, size_t *spatial_bytes);
+
+/* Create a handle over caller-allocated cache buffers.  temporal_buf / spatial_buf are
+ * device pointers of at least the sizes above (spatial_buf may be NULL when P' = 0).
+ * Contents need no initialisation: the queue starts empty (head = count = 0).
+ * *out receives a host-allocated handle, released with ca2_cache_destroy. */
+int ca2_cache_init(const ca2_config *cfg, void *temporal_buf, size_t temporal_bytes,
+                   void *spatial_buf, size_t spatial_bytes, ca2_cache **out);
+
+/* Release the handle (not the caller's buffers).  NULL is accepted. */
+int ca2_cache_destroy(ca2_cache *cache);
+
+/* Dequeue the n oldest queued frames (papernotes page, 关键设计 4: once the queue reaches
+ * Pmax the earliest cache entries leave it).  Host-only: head = (head + n) mod Pmax,
+ * count -= n.  0 <= n <= count, else CA2_ERR_CAPACITY. */
+int ca2_cache_evict(ca2_cache *cache, int n_frames);
+
+/* Cache-writing stage (papernotes page, 整体框架 and 关键设计 4-5).  For every layer L:
+ * frames j = 0..n-1 of k_t[L], v_t[L] ([B][n][HW][H][D]) are copied into ring slots
+ * (head + count + j) mod Pmax; then the spatial cache of layer L is overwritten with the
+ * last min(P', n) frames of k_s[L], v_s[L].  count += n.  One kernel launch for all
+ * layers; a bit-exact copy.  k_t, v_t, k_s, v_s are HOST arrays of N_L device pointers
+ * (k_s, v_s may be NULL when P' = 0).  1 <= n <= l; count + n > Pmax is
+ * CA2_ERR_CAPACITY (evict first). */
+int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const *v_t,
+                    const void *const *k_s, const void *const *v_s, int n_frames, void *stream);
+
+/* Causal temporal attention of one layer (papernotes page, 关键设计 1, equation
+ * CausalAttn; bohrium arXiv 2411.16375 page, formula with M_ij = -inf for i < j).
+ * For every (b, s, h) and chunk frame c:
+ *   out[b][c][s][h] = sum_j softmax_j(q . k_j / sqrt(D)) v_j
+ * over the keys j = the count queued frames (oldest first) followed by chunk frames
+ * 0..c of k, v.  The cache is only read.  q, k, v, out: [B][n][HW][H][D] device
+ * pointers; out must not overlap the inputs.  1 <= n <= l.  fp32 softmax and
+ * accumulation, bf16 output (round to nearest even). */
+int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k, const void *v,
+                      void *out, int n_frames, void *stream);
+
+/* Prefix-enhanced spatial attention of one layer (papernotes page, 关键设计 3).  For every
+ * (b, frame f, h) and token i:
+ *   out[b][f][i][h] = sum_j softmax_j(q_i . k_j / sqrt(D)) v_j
+ * use_prefix = 1 (denoising targets): keys/values are frame f's own HW tokens followed
+ *   by the HW tokens of each of the sp_count spatial-cache frames, an attention map of
+ *   HW x ((1 + sp_count) HW).
+ * use_prefix = 0 (clean prefix frames, the cache-writing pass): keys/values are frame f's
+ *   own tokens repeated P'+1 times; repetition leaves softmax attention unchanged, so
+ *   the kernel reads them once.
+ * q, k, v, out: [B][n][HW][H][D]; 1 <= n <= l. */
+int ca2_spatial_prefix_attn(ca2_cache *cache, int layer, const void *q, const void *k,
+                            const void *v, void *out, int n_frames, int use_prefix, void *stream);
+
+/* Cyclic temporal positional-embedding indices (papernotes page, 关键设计 4, Cyclic-TPEs):
+ * out_host[c] = (offset + first_global_frame + c) mod N_tpe for c < n.  Host-only.
+ * first_global_frame >= 0, offset >= 0, n >= 0; out_host may be NULL only when n = 0. */
+int ca2_tpe_indices(const ca2_cache *cache, long long first_global_frame, int offset, int n,
+                    int *out_host);
+
+/* Queue state: ring slot of the oldest frame, queued frames, spatial frames, and the
+ * total number of frames ever written.  Any out pointer may be NULL. */
+int ca2_cache_state(const ca2_cache *cache, int *head, int *count, int *sp_count,
+                    long long *frames_written);
+
+/* Synchronise the current device and return CA2_ERR_TIMEOUT if any kernel of this library
+ * recorded a bounded wait that gave up since the last call (clearing the record), else
+ * CA2_OK (or CA2_ERR_CUDA if the synchronisation itself fails). */
+int ca2_device_status(void);
+
+/* Self-test of the bounded-wait path: launches one block that waits on a barrier nothing
+ * will ever complete, with a wait limit of about wait_us microseconds; the kernel gives up,
+ * records the timeout and returns.  Follow with ca2_device_status, which must report
+ * CA2_ERR_TIMEOUT.  1 <= wait_us <= 1000000. */
+int ca2_selftest_timeout(int wait_us, void *stream);
+
+/* Static description of an error code. */
+const char *ca2_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CA2_H */

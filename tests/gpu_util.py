@@ -1,0 +1,159 @@
+"""Helpers for GPU parity tests: bf16 bit transfers, the tolerance check, and a driver that
+runs the Ca2-VDM generation loop through the C ABI next to the CPU oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from ca2_synth import Generator, Workload, bf16_to_f32
+
+# Tolerance for floating-point outputs (bf16 inputs, fp32 softmax and accumulation,
+# bf16 output): relative L2 5e-3, and max-abs 2e-2 on the error beyond the output format's
+# own rounding radius.  The outputs are bf16 by contract, and bf16 rounding alone moves a
+# value of magnitude in [2^e, 2^(e+1)) by up to 2^(e-8) (0.0156 in [4, 8), 0.031 in
+# [8, 16)), which no bf16-output kernel can avoid; that radius is taken off before the
+# max-abs bound applies.  Values below 1 in magnitude have a radius under 0.002.
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Rounding radius of bf16 (8 significant bits) at each value: 2^(floor(log2|x|) - 8)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
+def to_dev(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_bits(t) -> np.ndarray:
+    import torch
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def check_close(got_bits: np.ndarray, ref: np.ndarray, what: str = ""):
+    """Returns (raw max-abs, max-abs beyond the bf16 output rounding, rel-L2)."""
+    got = bf16_to_f32(got_bits).astype(np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), "%s: non-finite output" % what
+    err = np.abs(got - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    excess = float((err - bf16_half_ulp(ref)).max()) if err.size else 0.0
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    assert excess <= MAX_ABS and rel <= REL_L2, \
+        "%s: max-abs %.3g (beyond bf16 output rounding %.3g) rel-L2 %.3g" % (what, max_abs, excess, rel)
+    return max_abs, excess, rel
+
+
+class Loop:
+    """Drive one layer-stack of the AR loop on the GPU and mirror it in the oracle."""
+
+    def __init__(self, wl: Workload, seed: int = 0, tpe_offset: int = 0):
+        import torch
+        from causal_kv_cache_b200.ca2 import KVCache
+        self.torch = torch
+        self.wl = wl
+        self.gen = Generator(wl, seed)
+        self.cache = KVCache(wl.n_layers, wl.batch, wl.hw, wl.heads, wl.head_dim, wl.chunk_len,
+                             wl.p_max, wl.p_spatial)
+        self.rings = [oracle.RingModel(wl.p_max, wl.p_spatial) for _ in range(wl.n_layers)]
+        self.tpe_offset = tpe_offset
+        self.stats = []
+
+    # -- one attention call on both sides ----------------------------------------------
+    def temporal(self, layer, q, k, v, units=None):
+        n = q.shape[1]
+        out = self.torch.empty(q.shape, dtype=self.torch.bfloat16, device="cuda")
+        self.cache.temporal(layer, to_dev(q), to_dev(k), to_dev(v), out, n)
+        got = to_bits(out)
+        pk, pv = self.rings[layer].prefix()
+        if units is None:
+            ref = oracle.temporal_attn(q, k, v, pk, pv)
+            self.stats.append(("temporal", len(pk), n) + check_close(got, ref, "temporal P_k=%d" % len(pk)))
+        else:
+            ref = oracle.temporal_attn(q, k, v, pk, pv, units=units)
+            wl = self.wl
+            g = got.transpose(0, 2, 3, 1, 4).reshape(wl.batch * wl.hw * wl.heads, n, wl.head_dim)[units]
+            self.stats.append(("temporal", len(pk), n) + check_close(g, ref, "temporal(sampled)"))
+        return got
+
+    def spatial(self, layer, q, k, v, use_prefix, units=None):
+        n = q.shape[1]
+        out = self.torch.empty(q.shape, dtype=self.torch.bfloat16, device="cuda")
+        self.cache.spatial_attn(layer, to_dev(q), to_dev(k), to_dev(v), out, n, use_prefix)
+        got = to_bits(out)
+        if use_prefix:
+            sk, sv = self.rings[layer].spatial()
+            rep = 0
+        else:
+            sk, sv, rep = [], [], self.wl.p_spatial + 1
+        if units is None:
+            ref = oracle.spatial_attn(q, k, v, sk, sv, repeat=rep)
+            self.stats.append(("spatial", len(sk), n) + check_close(got, ref, "spatial n_sp=%d" % len(sk)))
+        else:
+            ref = oracle.spatial_attn(q, k, v, sk, sv, repeat=rep, units=units)
+            wl = self.wl
+            g = got.transpose(0, 1, 3, 2, 4).reshape(wl.batch * n * wl.heads, wl.hw, wl.head_dim)[units]
+            self.stats.append(("spatial", len(sk), n) + check_close(g, ref, "spatial(sampled)"))
+        return got
+
+    # -- cache-writing stage ------------------------------------------------------------
+    def write(self, kts, vts, kss, vss):
+        n = kts[0].shape[1]
+        e = self.cache.evict_for(n)
+        self.cache.write([to_dev(x) for x in kts], [to_dev(x) for x in vts],
+                         [to_dev(x) for x in kss], [to_dev(x) for x in vss], n)
+        for L in range(self.wl.n_layers):
+            gone = self.rings[L].write(kts[L], vts[L], kss[L], vss[L])
+            assert len(gone) == e
+        self.check_cache_bits()
+
+    def check_cache_bits(self):
+        """Ring slots and spatial cache against the oracle's frames, bit for bit."""
+        self.torch.cuda.synchronize()
+        head, count, sp, fw = self.cache.state()
+        for L, ring in enumerate(self.rings):
+            assert (head, count, sp, fw) == (ring.head, ring.count, len(ring.spatial_ids), ring.frames_written)
+            rk = to_bits(self.cache.ring(L, 0))
+            rv = to_bits(self.cache.ring(L, 1))
+            for g in ring.queue:
+                slot = ring.slot_of(g)
+                assert np.array_equal(rk[slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rv[slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
+            if self.wl.p_spatial:
+                sk = to_bits(self.cache.spatial(L, 0))
+                sv = to_bits(self.cache.spatial(L, 1))
+                for j, g in enumerate(ring.spatial_ids):
+                    assert np.array_equal(sk[j], ring.sk[g]) and np.array_equal(sv[j], ring.sv[g])
+
+    def tpe_check(self, n):
+        g0 = self.rings[0].frames_written
+        got = self.cache.tpe(g0, self.tpe_offset, n)
+        assert got == oracle.tpe_indices(g0, self.tpe_offset, n, self.wl.tpe_len)
+        return got
+
+    # -- whole passes ------------------------------------------------------------------
+    def pass_(self, n, use_prefix, t_units=None, s_units=None):
+        """One forward pass over all layers: spatial then temporal attention per layer."""
+        outs = []
+        for L in range(self.wl.n_layers):
+            sq, sk_, sv_ = self.gen.qkv(n)
+            tq, tk, tv = self.gen.qkv(n)
+            so = self.spatial(L, sq, sk_, sv_, use_prefix, units=s_units)
+            to = self.temporal(L, tq, tk, tv, units=t_units)
+            outs.append((sk_, sv_, tk, tv, so, to))
+        return outs
+
+    def ar_step(self, n, T, t_units=None, s_units=None):
+        self.tpe_check(n)
+        for _ in range(T):
+            self.pass_(n, 1, t_units, s_units)
+        outs = self.pass_(n, 0, t_units, s_units)   # cache-writing pass (clean chunk)
+        self.write([o[2] for o in outs], [o[3] for o in outs], [o[0] for o in outs], [o[1] for o in outs])
+
+    def first_frame(self):
+        outs = self.pass_(1, 0)
+        self.write([o[2] for o in outs], [o[3] for o in outs], [o[0] for o in outs], [o[1] for o in outs])

@@ -1,0 +1,167 @@
+"""The C ABI of libca2.so on the host: exports, validation and host-only state (no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from causal_kv_cache_b200 import ca2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE_T = 0x7F0000000000          # 16-byte aligned stand-ins; never dereferenced on the host
+FAKE_S = 0x7F1000000000
+
+
+def cfg(**kw):
+    base = dict(n_layers=1, batch=1, hw=256, heads=16, head_dim=72, chunk_len=8, p_max=41,
+                p_spatial=3, tpe_len=0)
+    base.update(kw)
+    return base
+
+
+def make(**kw):
+    c = cfg(**kw)
+    tb, sb = ca2.ca2_cache_bytes(c)
+    return ca2.ca2_cache_init(c, FAKE_T, tb, FAKE_S if sb else None, sb), c
+
+
+def test_library_exports_every_declared_symbol():
+    with open(os.path.join(ROOT, "include", "ca2.h")) as f:
+        header = f.read()
+    declared = set(re.findall(r"^(?:int|const char \*)\s*(ca2_\w+)\s*\(", header, re.M))
+    assert {"ca2_cache_init", "ca2_cache_write", "ca2_temporal_attn", "ca2_spatial_prefix_attn",
+            "ca2_cache_evict"} <= declared
+    lib = ctypes.CDLL(ca2.LIBRARY_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert set(ca2.__all__) >= declared
+
+
+def test_cache_bytes_matches_oracle_and_memory_table():
+    for kw in (dict(), dict(n_layers=28, batch=4, p_max=41), dict(n_layers=28, p_max=25),
+               dict(hw=16, heads=2, head_dim=16, chunk_len=4, p_max=9, p_spatial=1)):
+        c = cfg(**kw)
+        t, s = ca2.ca2_cache_bytes(c)
+        assert t + s == oracle.cache_bytes(c["n_layers"], c["batch"], c["hw"], c["heads"], c["head_dim"],
+                                           c["p_max"], c["p_spatial"])
+        assert s == oracle.cache_bytes(c["n_layers"], c["batch"], c["hw"], c["heads"], c["head_dim"], 0,
+                                       c["p_spatial"])
+    # the Ca2-VDM memory-table setting: 0.86 GiB with prefix enhancement
+    t, s = ca2.ca2_cache_bytes(cfg(n_layers=28, p_max=25))
+    assert t + s == 924_844_032
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(head_dim=12), -2), (dict(head_dim=136), -2), (dict(head_dim=0), -2),
+    (dict(chunk_len=9), -2), (dict(chunk_len=0), -2), (dict(p_max=7), -2),
+    (dict(p_spatial=9), -2), (dict(p_spatial=-1), -2), (dict(n_layers=0), -2),
+    (dict(batch=0), -2), (dict(hw=0), -2), (dict(heads=0), -2), (dict(tpe_len=-1), -2),
+])
+def test_invalid_configs_rejected(bad, code):
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_bytes(cfg(**bad))
+    assert e.value.status == code
+
+
+def test_init_validation():
+    c = cfg()
+    tb, sb = ca2.ca2_cache_bytes(c)
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_init(c, FAKE_T, tb - 1, FAKE_S, sb)
+    assert e.value.status == -3
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_init(c, FAKE_T, tb, FAKE_S, sb - 16)
+    assert e.value.status == -3
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_init(c, FAKE_T + 8, tb, FAKE_S, sb)
+    assert e.value.status == -4
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_init(c, None, tb, FAKE_S, sb)
+    assert e.value.status == -1
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_init(c, FAKE_T, tb, None, sb)
+    assert e.value.status == -1
+    # P' = 0 needs no spatial buffer
+    c0 = cfg(p_spatial=0)
+    tb0, sb0 = ca2.ca2_cache_bytes(c0)
+    assert sb0 == 0
+    h = ca2.ca2_cache_init(c0, FAKE_T, tb0, None, 0)
+    ca2.ca2_cache_destroy(h)
+    ca2.ca2_cache_destroy(None)
+
+
+def test_fresh_state_and_evict_bounds():
+    h, c = make()
+    assert ca2.ca2_cache_state(h) == (0, 0, 0, 0)
+    ca2.ca2_cache_evict(h, 0)
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_evict(h, 1)
+    assert e.value.status == -3
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_evict(h, -1)
+    assert e.value.status == -3
+    ca2.ca2_cache_destroy(h)
+
+
+def test_call_validation_before_any_launch():
+    h, c = make()
+    al = 0x7E0000000000
+    # temporal / spatial argument checks
+    for fn in (lambda *a: ca2.ca2_temporal_attn(h, *a, stream=0),
+               lambda *a: ca2.ca2_spatial_prefix_attn(h, *a, 1, stream=0)):
+        with pytest.raises(ca2.Ca2Error) as e:
+            fn(1, al, al, al, al, 8)
+        assert e.value.status == -1          # layer out of range
+        with pytest.raises(ca2.Ca2Error) as e:
+            fn(0, None, al, al, al, 8)
+        assert e.value.status == -1
+        with pytest.raises(ca2.Ca2Error) as e:
+            fn(0, al, al, al, al, 9)
+        assert e.value.status == -2          # more frames than the chunk length
+        with pytest.raises(ca2.Ca2Error) as e:
+            fn(0, al, al, al, al, 0)
+        assert e.value.status == -2
+        with pytest.raises(ca2.Ca2Error) as e:
+            fn(0, al + 2, al, al, al, 8)
+        assert e.value.status == -4
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_spatial_prefix_attn(h, 0, al, al, al, al, 8, 2, stream=0)
+    assert e.value.status == -1
+    # cache write checks: shape, missing spatial tensors, alignment, capacity
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_write(h, [al], [al], [al], [al], 9, stream=0)
+    assert e.value.status == -2
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_write(h, [al], [al], None, None, 8, stream=0)
+    assert e.value.status == -1
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_write(h, [al + 4], [al], [al], [al], 8, stream=0)
+    assert e.value.status == -4
+    ca2.ca2_cache_destroy(h)
+    # capacity: Pmax = 8 = l; a full chunk fits once, the next needs eviction first
+    h2, _ = make(p_max=8)
+    with pytest.raises(ca2.Ca2Error):
+        ca2.ca2_cache_write(h2, [al], [al], [al], [al], 9, stream=0)
+    ca2.ca2_cache_destroy(h2)
+
+
+def test_tpe_indices_match_oracle():
+    h, c = make()
+    n_tpe = c["p_max"] + c["chunk_len"]       # tpe_len 0 selects Pmax + l
+    for g0 in (0, 1, 41, 45, 49, 1000, 10 ** 12):
+        for off in (0, 7, 48):
+            assert ca2.ca2_tpe_indices(h, g0, off, 8) == oracle.tpe_indices(g0, off, 8, n_tpe)
+    assert ca2.ca2_tpe_indices(h, 5, 0, 0) == []
+    with pytest.raises(ca2.Ca2Error):
+        ca2.ca2_tpe_indices(h, -1, 0, 1)
+    ca2.ca2_cache_destroy(h)
+    h, c = make(tpe_len=16)
+    assert ca2.ca2_tpe_indices(h, 14, 1, 4) == oracle.tpe_indices(14, 1, 4, 16)
+    ca2.ca2_cache_destroy(h)
+
+
+def test_status_strings():
+    for code in range(-6, 1):
+        assert ca2.ca2_status_string(code) != "unknown status"
+    assert ca2.ca2_status_string(-99) == "unknown status"
