@@ -49,11 +49,14 @@ _lib = None
 
 
 def load_library(path: Optional[str] = None):
-    """Load libca2.so (no fallback: a missing library is an error)."""
+    """Load libca2.so (no fallback: a missing library is an error).
+
+    The environment variable CA2_LIBRARY, when set, names another build of the library
+    to load instead of the in-tree one."""
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIBRARY_PATH
+    p = path or os.environ.get("CA2_LIBRARY") or LIBRARY_PATH
     if not os.path.exists(p):
         raise RuntimeError("libca2.so is not built (%s); run `python -m causal_kv_cache_b200.build`" % p)
     lib = ctypes.CDLL(p)
@@ -213,8 +216,8 @@ def ca2_status_string(status: int) -> str:
 class KVCache:
     """Cache buffers allocated with torch on the current CUDA device, plus the handle.
 
-    ``ring(layer, kv)`` and ``spatial(layer, kv)`` are bf16 views of the buffers with the
-    layout documented in include/ca2.h ([Pmax or P'][B][HW][H][D]).
+    ``ring(layer, kv)`` ([B][HW][Pmax][H][D]) and ``spatial(layer, kv)`` ([P'][B][HW][H][D])
+    are bf16 views of the buffers with the layout documented in include/ca2.h.
     """
 
     def __init__(self, n_layers, batch, hw, heads, head_dim, chunk_len, p_max, p_spatial,
@@ -239,10 +242,11 @@ class KVCache:
             pass
 
     def ring(self, layer: int, kv: int):
+        """Token-major ring of one layer: [B][HW][Pmax][H][D]."""
         c = self.cfg
         per = c.p_max * c.batch * c.hw * c.heads * c.head_dim
         off = (layer * 2 + kv) * per
-        return self.tbuf[off:off + per].view(c.p_max, c.batch, c.hw, c.heads, c.head_dim)
+        return self.tbuf[off:off + per].view(c.batch, c.hw, c.p_max, c.heads, c.head_dim)
 
     def spatial(self, layer: int, kv: int):
         c = self.cfg

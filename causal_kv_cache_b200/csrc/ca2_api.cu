@@ -13,12 +13,12 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
-#include "../../include/ca2.h"
+#include "ca2.h"
 #include "ca2_kernels.h"
 
 struct ca2_cache {
     ca2_config cfg;
-    uint8_t *tbuf;      // [N_L][2][Pmax][B][HW][H][D] bf16
+    uint8_t *tbuf;      // [N_L][2][B][HW][Pmax][H][D] bf16 (token-major ring)
     uint8_t *sbuf;      // [N_L][2][P'][B][HW][H][D] bf16
     size_t plane_bytes; // bytes of one frame-plane B*HW*H*D*2
     int head;           // ring slot of the oldest queued frame
@@ -37,7 +37,7 @@ int validate_config(const ca2_config *c)
     if (c->n_layers < 1 || c->batch < 1 || c->hw < 1 || c->heads < 1) return CA2_ERR_SHAPE;
     if (c->head_dim < 8 || c->head_dim > 128 || (c->head_dim % 8) != 0) return CA2_ERR_SHAPE;
     if (c->chunk_len < 1 || c->chunk_len > ca2::kMaxChunk) return CA2_ERR_SHAPE;
-    if (c->p_max < c->chunk_len) return CA2_ERR_SHAPE;
+    if (c->p_max < c->chunk_len || c->p_max > ca2::kMaxRingSlots) return CA2_ERR_SHAPE;
     if (c->p_spatial < 0 || c->p_spatial > c->chunk_len) return CA2_ERR_SHAPE;
     if (c->tpe_len < 0) return CA2_ERR_SHAPE;
     // tensor-map extents and 32-bit strides
@@ -92,6 +92,24 @@ bool encode_4d(CUtensorMap *m, const void *base, int D, int H, int HW, int frame
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 5-D view (D, frames, H, HW, B) of a bf16 tensor with the given frame, token and video
+// strides (elements; heads are D apart); box D x box_frames x box_heads x 1 x 1, no swizzle.
+bool encode_5d(CUtensorMap *m, const void *base, int D, int frames, int H, int HW, int B, long long frame_stride,
+               long long token_stride, long long video_stride, int box_frames, int box_heads)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)frames, (cuuint64_t)H, (cuuint64_t)HW, (cuuint64_t)B};
+    cuuint64_t strides[4] = {(cuuint64_t)frame_stride * 2, (cuuint64_t)D * 2, (cuuint64_t)token_stride * 2,
+                             (cuuint64_t)video_stride * 2};
+    cuuint32_t box[5] = {(cuuint32_t)D, (cuuint32_t)box_frames, (cuuint32_t)box_heads, 1u, 1u};
+    cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -194,9 +212,10 @@ int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t
     std::memset(&p, 0, sizeof(p));
     p.tbuf = reinterpret_cast<uint4 *>(c->tbuf);
     p.sbuf = reinterpret_cast<uint4 *>(c->sbuf);
-    p.plane_vec = (long long)(c->plane_bytes / (size_t)g.batch / 16u);
+    p.row_vec = (long long)g.heads * g.head_dim / 8;   // 16-byte vectors per (video, token, frame) row
+    p.tokens = (long long)g.batch * g.hw;
+    p.hw = g.hw;
     p.n = n;
-    p.B = g.batch;
     p.slot0 = (c->head + c->count) % g.p_max;
     p.p_max = g.p_max;
     p.n_sp = n_sp;
@@ -227,12 +246,7 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
     if (st != CA2_OK) return st;
     const ca2_config &g = c->cfg;
     ca2::TemporalParams p;
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
     p.out = static_cast<__nv_bfloat16 *>(out);
-    p.ring_k = reinterpret_cast<const __nv_bfloat16 *>(layer_ring(c, layer, 0));
-    p.ring_v = reinterpret_cast<const __nv_bfloat16 *>(layer_ring(c, layer, 1));
     p.B = g.batch;
     p.HW = g.hw;
     p.H = g.heads;
@@ -245,15 +259,27 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
     while (g.heads % G) G >>= 1;
     p.G = G;
     p.n_items = g.batch * g.hw * (g.heads / G);
-    p.n_stages = (c->count + n + 15) / 16;
+    p.ring_box_mask = 0;
+    for (int i = 0; i < c->count; ++i) p.ring_box_mask |= 1u << (((c->head + i) % g.p_max) / 16);
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
-    p.row_bytes = (uint32_t)(G * g.head_dim * 2);
-    p.pitch = ca2::temporal_pitch(G, g.head_dim);
+
+    // temporal tensors are token-major: chunk [B][HW][n][C], ring [B][HW][Pmax][C], C = H*D
+    const long long C = (long long)g.heads * g.head_dim;
+    ca2::TemporalMaps m;
+    const bool ok =
+        encode_5d(&m.q, q, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 8, G) &&
+        encode_5d(&m.k, k, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 16, G) &&
+        encode_5d(&m.v, v, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 16, G) &&
+        encode_5d(&m.rk, layer_ring(c, layer, 0), g.head_dim, g.p_max, g.heads, g.hw, g.batch, C, g.p_max * C,
+                  (long long)g.hw * g.p_max * C, 16, G) &&
+        encode_5d(&m.rv, layer_ring(c, layer, 1), g.head_dim, g.p_max, g.heads, g.hw, g.batch, C, g.p_max * C,
+                  (long long)g.hw * g.p_max * C, 16, G);
+    if (!ok) return CA2_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return CA2_ERR_CUDA;
     int grid = 2 * sms;
     if (grid > p.n_items) grid = p.n_items;
-    return cuda_status(ca2::launch_temporal(p, grid, static_cast<cudaStream_t>(stream)));
+    return cuda_status(ca2::launch_temporal(m, p, grid, static_cast<cudaStream_t>(stream)));
 }
 
 int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *k, const void *v, void *out,
@@ -266,17 +292,26 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     const int n_sp = use_prefix ? c->sp_count : 0;
     const int frames = g.batch * n;
     ca2::SpatialMaps m;
-    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_32B;
-    bool ok = encode_4d(&m.q, q, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
-              encode_4d(&m.k, k, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
-              encode_4d(&m.v, v, g.head_dim, g.heads, g.hw, frames, 16, 128, sw) &&
-              encode_4d(&m.o, out, g.head_dim, g.heads, g.hw, frames, g.head_dim, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    const int D = g.head_dim, H = g.heads, HW = g.hw;
+    // wide boxes exist only when D >= 64; otherwise slot [0] is a copy that is never read
+    auto pair = [&](CUtensorMap *mm, const void *base, int frames_) {
+        if (!encode_4d(&mm[1], base, D, H, HW, frames_, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+        if (D < 64) {
+            mm[0] = mm[1];
+            return true;
+        }
+        return encode_4d(&mm[0], base, D, H, HW, frames_, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    bool ok = pair(m.q, q, frames) && pair(m.k, k, frames) && pair(m.v, v, frames) &&
+              encode_4d(&m.o, out, D, H, HW, frames, D, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && n_sp > 0) {
-        ok = encode_4d(&m.sk, layer_spatial(c, layer, 0), g.head_dim, g.heads, g.hw, n_sp * g.batch, 16, 128, sw) &&
-             encode_4d(&m.sv, layer_spatial(c, layer, 1), g.head_dim, g.heads, g.hw, n_sp * g.batch, 16, 128, sw);
+        ok = pair(m.sk, layer_spatial(c, layer, 0), n_sp * g.batch) &&
+             pair(m.sv, layer_spatial(c, layer, 1), n_sp * g.batch);
     } else if (ok) {
-        m.sk = m.k;   // never read when there is no prefix
-        m.sv = m.v;
+        for (int i = 0; i < 2; ++i) {   // never read when there is no prefix
+            m.sk[i] = m.k[i];
+            m.sv[i] = m.v[i];
+        }
     }
     if (!ok) return CA2_ERR_CUDA;
     ca2::SpatialParams p;

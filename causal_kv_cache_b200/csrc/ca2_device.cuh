@@ -91,6 +91,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int sit
     }
 }
 
+// Warp-wide wait: every lane polls (so every lane acquires the phase), and the outcome
+// is made uniform so that a warp never splits on a timeout.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int site, volatile int *abort)
+{
+    const bool ok = mbar_wait(bar, parity, site, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // ---- bulk copies (TMA engine) --------------------------------------------------------
 // 1-D bulk copy global -> shared, completing `bytes` of transaction on an mbarrier.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)

@@ -13,10 +13,7 @@ constexpr int kMaxTemporalGroup = 4;   // heads per work item = consumer warps p
 constexpr int kMaxChunk = 8;           // queries per (token, head): the chunk length limit
 
 struct TemporalParams {
-    const __nv_bfloat16 *q, *k, *v;     // chunk tensors [B][n][HW][H][D]
     __nv_bfloat16 *out;                 // [B][n][HW][H][D]
-    const __nv_bfloat16 *ring_k;        // this layer's K ring [Pmax][B][HW][H][D]
-    const __nv_bfloat16 *ring_v;        // this layer's V ring
     int B, HW, H, D;
     int n;          // chunk frames in this call (queries per token-head)
     int Pk;         // queued frames
@@ -24,15 +21,20 @@ struct TemporalParams {
     int Pmax;
     int G;          // heads per work item
     int n_items;    // B * HW * (H / G)
-    int n_stages;   // ceil((Pk + n) / 16)
-    float scale_log2;   // log2(e) / sqrt(D)
-    uint32_t row_bytes; // G * D * 2
-    uint32_t pitch;     // shared-memory row pitch
+    uint32_t ring_box_mask;   // bit i: ring slots [16i, 16i+16) hold at least one queued frame
+    float scale_log2;         // log2(e) / sqrt(D)
 };
 
-uint32_t temporal_pitch(int G, int D);
+// 5-D views (head dim, frame, head, token, video) of the chunk tensors and of one
+// layer's K and V rings; boxes of D x 16 frames x G heads (D x 8 x G for q).
+struct TemporalMaps {
+    CUtensorMap q, k, v, rk, rv;
+};
+
+constexpr int kMaxRingSlots = 16 * 32;   // the ring-box mask has 32 bits
+
 uint32_t temporal_smem_bytes(int G, int D);
-cudaError_t launch_temporal(const TemporalParams &p, int grid, cudaStream_t stream);
+cudaError_t launch_temporal(const TemporalMaps &m, const TemporalParams &p, int grid, cudaStream_t stream);
 
 // ---- cache write ------------------------------------------------------------------------
 constexpr int kMaxLayersPerWrite = 64;
@@ -43,13 +45,14 @@ struct CacheWriteLayer {
 
 struct CacheWriteParams {
     CacheWriteLayer layer[kMaxLayersPerWrite];
-    uint4 *tbuf;            // temporal cache base [N_L][2][Pmax][B][plane]
-    uint4 *sbuf;            // spatial cache base  [N_L][2][P'][B][plane]
-    long long plane_vec;    // 16-byte vectors per (video, frame) plane: HW*H*D/8
+    uint4 *tbuf;            // temporal cache base [N_L][2][B][HW][Pmax][C] (token-major ring)
+    uint4 *sbuf;            // spatial cache base  [N_L][2][P'][B][HW][C]
+    long long row_vec;      // 16-byte vectors per row of C = H*D elements
+    long long tokens;       // B * HW
+    int hw;
     int layer0;             // absolute index of layer[0]
     int n_layers;           // layers in this launch
     int n;                  // frames written
-    int B;
     int slot0;              // ring slot of frame 0: (head + count) mod Pmax
     int p_max;
     int n_sp;               // spatial frames written: min(P', n)
@@ -67,8 +70,10 @@ struct SpatialParams {
     float scale_log2;
 };
 
+// Loaded tensors have two maps each: [0] boxes of 64 head-dims x 128 tokens (128-byte
+// swizzle), [1] boxes of 16 head-dims x 128 tokens (32-byte swizzle).  o: D x 128 tokens.
 struct SpatialMaps {
-    CUtensorMap q, k, v, sk, sv, o;
+    CUtensorMap q[2], k[2], v[2], sk[2], sv[2], o;
 };
 
 uint32_t spatial_smem_bytes(int D);

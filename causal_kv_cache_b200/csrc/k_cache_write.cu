@@ -3,8 +3,9 @@
 // Ca2-VDM ("Ca2-VDM" papernotes page, 整体框架 and 关键设计 4-5): after a chunk is denoised,
 // one clean forward pass computes its K/V, which join the temporal queue (FIFO, at most
 // Pmax frames) and replace the one-chunk spatial cache.  This kernel is the data movement
-// of that step for every layer at once: a bit-exact copy of frame-planes, 16 bytes per
-// access, one block row per (layer, tensor, video, frame) copy.
+// of that step for every layer at once: a bit-exact copy, 16 bytes per access.  The ring
+// is token-major (each token's Pmax slots are contiguous), so a temporal write moves the
+// chunk's n rows of every token into that token's slots.
 #include <cstdint>
 
 #include "ca2_device.cuh"
@@ -28,55 +29,68 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 }
 }  // namespace
 
+// blockIdx.y = (layer, tensor): tensor 0/1 = temporal K/V, 2/3 = spatial K/V.
+//   temporal: chunk [B][HW][n][C] -> ring [B][HW][Pmax][C]; row (token, j) -> slot (slot0 + j) mod Pmax
+//   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
-    // blockIdx.y enumerates copies: per layer, B * (2n + 2 n_sp) of them
-    const int per_layer = p.B * (2 * p.n + 2 * p.n_sp);
-    const int cy = blockIdx.y;
-    const int li = cy / per_layer;
-    const int r = cy - li * per_layer;
-    const int t = r / p.B;          // which frame of which tensor
-    const int b = r - t * p.B;
+    const int li = blockIdx.y >> 2;
+    const int tensor = blockIdx.y & 3;
     const CacheWriteLayer &Ly = p.layer[li];
-    const int layer = p.layer0 + li;
-
+    const long long layer = p.layer0 + li;
+    const long long rv = p.row_vec;
+    long long total;
     const uint4 *src;
     uint4 *dst;
-    if (t < 2 * p.n) {
-        const int kv = t >= p.n;
-        const int j = kv ? t - p.n : t;
-        int slot = p.slot0 + j;
-        if (slot >= p.p_max) slot -= p.p_max;
-        src = (kv ? Ly.vt : Ly.kt) + ((long long)b * p.n + j) * p.plane_vec;
-        dst = p.tbuf + ((((long long)layer * 2 + kv) * p.p_max + slot) * p.B + b) * p.plane_vec;
+    if (tensor < 2) {
+        total = p.tokens * p.n * rv;
+        src = tensor == 0 ? Ly.kt : Ly.vt;
+        dst = p.tbuf + ((layer * 2 + tensor) * p.tokens) * p.p_max * rv;
     } else {
-        const int u = t - 2 * p.n;
-        const int kv = u >= p.n_sp;
-        const int jsp = kv ? u - p.n_sp : u;             // spatial slot, oldest first
-        const int j = p.n - p.n_sp + jsp;                // frame of the chunk
-        src = (kv ? Ly.vs : Ly.ks) + ((long long)b * p.n + j) * p.plane_vec;
-        dst = p.sbuf + ((((long long)layer * 2 + kv) * p.p_spatial + jsp) * p.B + b) * p.plane_vec;
+        total = (long long)p.n_sp * p.tokens * rv;
+        src = tensor == 2 ? Ly.ks : Ly.vs;
+        dst = p.sbuf + ((layer * 2 + (tensor - 2)) * p.p_spatial) * p.tokens * rv;
     }
-
     const long long base = (long long)blockIdx.x * (kThreads * kVecPerThread) + threadIdx.x;
+    if (base >= total) return;
     uint4 v[kVecPerThread];
+    long long so[kVecPerThread], dof[kVecPerThread];
 #pragma unroll
     for (int i = 0; i < kVecPerThread; ++i) {
         const long long e = base + (long long)i * kThreads;
-        if (e < p.plane_vec) v[i] = ld_stream(src + e);
+        so[i] = dof[i] = -1;
+        if (e < total) {
+            const long long row = e / rv, off = e - row * rv;
+            if (tensor < 2) {
+                const long long tok = row / p.n;
+                const int j = (int)(row - tok * p.n);
+                int slot = p.slot0 + j;
+                if (slot >= p.p_max) slot -= p.p_max;
+                so[i] = e;
+                dof[i] = (tok * p.p_max + slot) * rv + off;
+            } else {
+                // row = jsp * tokens + (b * HW + s); source frame n - n_sp + jsp of video b
+                const long long jsp = row / p.tokens;
+                const long long bt = row - jsp * p.tokens;
+                const long long b = bt / p.hw, sidx = bt - b * p.hw;
+                so[i] = ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * rv + off;
+                dof[i] = e;
+            }
+            v[i] = ld_stream(src + so[i]);
+        }
     }
 #pragma unroll
-    for (int i = 0; i < kVecPerThread; ++i) {
-        const long long e = base + (long long)i * kThreads;
-        if (e < p.plane_vec) dst[e] = v[i];
-    }
+    for (int i = 0; i < kVecPerThread; ++i)
+        if (dof[i] >= 0) dst[dof[i]] = v[i];
 }
 
 cudaError_t launch_cache_write(const CacheWriteParams &p, cudaStream_t stream)
 {
     const long long per_block = (long long)kThreads * kVecPerThread;
-    dim3 grid((unsigned)((p.plane_vec + per_block - 1) / per_block),
-              (unsigned)(p.n_layers * p.B * (2 * p.n + 2 * p.n_sp)));
+    const long long t_total = p.tokens * p.n * p.row_vec;
+    const long long s_total = (long long)p.n_sp * p.tokens * p.row_vec;
+    const long long most = t_total > s_total ? t_total : s_total;
+    dim3 grid((unsigned)((most + per_block - 1) / per_block), (unsigned)(p.n_layers * 4));
     if (grid.x == 0 || grid.y == 0) return cudaSuccess;
     k_cache_write<<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();

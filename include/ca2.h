@@ -9,9 +9,12 @@
  * denoising step (prefix frames use tEmb(0)), so one copy serves all T steps.
  *
  * Conventions shared by every call:
- *   - Elements are bfloat16.  Chunk tensors (q, k, v, out) are dense, row-major
- *     [B][n][HW][H][D]: video, frame of the chunk, spatial token, head, head dim.
- *     All device pointers must be 16-byte aligned.
+ *   - Elements are bfloat16.  Spatial chunk tensors (q, k, v, out of the spatial call and
+ *     the k_s, v_s given to the cache write) are frame-major [B][n][HW][H][D]: video, frame
+ *     of the chunk, spatial token, head, head dim -- the (B*T) x S x C view a spatial block
+ *     works in.  Temporal chunk tensors (q, k, v, out of the temporal call and the k_t, v_t
+ *     given to the cache write) are token-major [B][HW][n][H][D] -- the (B*S) x T x C view a
+ *     temporal block works in.  All device pointers must be 16-byte aligned.
  *   - The caller owns all device memory (allocate it however you like, e.g. torch).
  *     The library stores the two cache pointers given to ca2_cache_init and never
  *     frees or reallocates them.
@@ -25,12 +28,13 @@
  *   - A handle is not thread-safe.
  *
  * Cache memory layout (both buffers caller-allocated, sizes from ca2_cache_bytes):
- *   temporal: [N_L][2][Pmax][B][HW][H][D]   (index 0 = K ring, 1 = V ring)
+ *   temporal: [N_L][2][B][HW][Pmax][H][D]   (index 0 = K ring, 1 = V ring; token-major:
+ *                                            a token's Pmax slots are contiguous)
  *   spatial : [N_L][2][P'][B][HW][H][D]
- * A ring slot is one frame-plane [B][HW][H][D] with exactly the layout of one frame of
- * a chunk tensor.  The i-th oldest queued frame (i = 0 .. count-1) is in slot
- * (head + i) mod Pmax; spatial slot j (j < sp_count) holds the j-th of the last
- * sp_count frames written, oldest first.
+ * The i-th oldest queued frame (i = 0 .. count-1) is in ring slot (head + i) mod Pmax;
+ * spatial slot j (j < sp_count) holds the j-th of the last sp_count frames written,
+ * oldest first.  Slots that hold no queued frame may contain anything: they are masked,
+ * and their values never reach an output.
  *
  * Required order within one AR step:
  *   T x { for each layer: ca2_spatial_prefix_attn(use_prefix=1), ca2_temporal_attn }
@@ -57,7 +61,7 @@ typedef struct {
     int heads;      /* H >= 1                                                              */
     int head_dim;   /* D: multiple of 8, 8 <= D <= 128                                     */
     int chunk_len;  /* l: frames per AR chunk, 1 <= l <= 8                                 */
-    int p_max;      /* Pmax >= l: capacity of the temporal queue, in frames                */
+    int p_max;      /* l <= Pmax <= 512: capacity of the temporal queue, in frames         */
     int p_spatial;  /* P': 0 <= P' <= l prefix frames kept for spatial attention           */
     int tpe_len;    /* N_tpe >= 1: temporal positional table length; 0 selects Pmax + l     */
 } ca2_config;
@@ -94,11 +98,12 @@ int ca2_cache_destroy(ca2_cache *cache);
 int ca2_cache_evict(ca2_cache *cache, int n_frames);
 
 /* Cache-writing stage (papernotes page, 整体框架 and 关键设计 4-5).  For every layer L:
- * frames j = 0..n-1 of k_t[L], v_t[L] ([B][n][HW][H][D]) are copied into ring slots
+ * frames j = 0..n-1 of k_t[L], v_t[L] are copied into ring slots
  * (head + count + j) mod Pmax; then the spatial cache of layer L is overwritten with the
  * last min(P', n) frames of k_s[L], v_s[L].  count += n.  One kernel launch for all
- * layers; a bit-exact copy.  k_t, v_t, k_s, v_s are HOST arrays of N_L device pointers
- * (k_s, v_s may be NULL when P' = 0).  1 <= n <= l; count + n > Pmax is
+ * layers; a bit-exact copy.  k_t[L], v_t[L] are token-major [B][HW][n][H][D]; k_s[L],
+ * v_s[L] are frame-major [B][n][HW][H][D].  k_t, v_t, k_s, v_s are HOST arrays of N_L
+ * device pointers (k_s, v_s may be NULL when P' = 0).  1 <= n <= l; count + n > Pmax is
  * CA2_ERR_CAPACITY (evict first). */
 int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const *v_t,
                     const void *const *k_s, const void *const *v_s, int n_frames, void *stream);
@@ -106,11 +111,12 @@ int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const 
 /* Causal temporal attention of one layer (papernotes page, 关键设计 1, equation
  * CausalAttn; bohrium arXiv 2411.16375 page, formula with M_ij = -inf for i < j).
  * For every (b, s, h) and chunk frame c:
- *   out[b][c][s][h] = sum_j softmax_j(q . k_j / sqrt(D)) v_j
- * over the keys j = the count queued frames (oldest first) followed by chunk frames
- * 0..c of k, v.  The cache is only read.  q, k, v, out: [B][n][HW][H][D] device
- * pointers; out must not overlap the inputs.  1 <= n <= l.  fp32 softmax and
- * accumulation, bf16 output (round to nearest even). */
+ *   out[b][s][c][h] = sum_j softmax_j(q[b][s][c][h] . k_j / sqrt(D)) v_j
+ * over the keys j = the count queued frames followed by chunk frames 0..c of k, v (the
+ * queued frames are all visible, so their order does not matter).  The cache is only
+ * read.  q, k, v, out: token-major [B][HW][n][H][D] device pointers; out must not
+ * overlap the inputs.  1 <= n <= l.  fp32 softmax and accumulation, bf16 output (round
+ * to nearest even). */
 int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k, const void *v,
                       void *out, int n_frames, void *stream);
 
@@ -123,7 +129,7 @@ int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k,
  * use_prefix = 0 (clean prefix frames, the cache-writing pass): keys/values are frame f's
  *   own tokens repeated P'+1 times; repetition leaves softmax attention unchanged, so
  *   the kernel reads them once.
- * q, k, v, out: [B][n][HW][H][D]; 1 <= n <= l. */
+ * q, k, v, out: frame-major [B][n][HW][H][D]; 1 <= n <= l. */
 int ca2_spatial_prefix_attn(ca2_cache *cache, int layer, const void *q, const void *k,
                             const void *v, void *out, int n_frames, int use_prefix, void *stream);
 

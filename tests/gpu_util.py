@@ -34,6 +34,11 @@ def to_bits(t) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def token_major(x: np.ndarray) -> np.ndarray:
+    """[B][n][HW][H][D] -> [B][HW][n][H][D] (the temporal tensors' layout)."""
+    return np.ascontiguousarray(np.swapaxes(x, 1, 2))
+
+
 def check_close(got_bits: np.ndarray, ref: np.ndarray, what: str = ""):
     """Returns (raw max-abs, max-abs beyond the bf16 output rounding, rel-L2)."""
     got = bf16_to_f32(got_bits).astype(np.float64)
@@ -65,10 +70,11 @@ class Loop:
 
     # -- one attention call on both sides ----------------------------------------------
     def temporal(self, layer, q, k, v, units=None):
+        """q, k, v frame-major [B][n][HW][H][D]; the GPU gets them token-major."""
         n = q.shape[1]
-        out = self.torch.empty(q.shape, dtype=self.torch.bfloat16, device="cuda")
-        self.cache.temporal(layer, to_dev(q), to_dev(k), to_dev(v), out, n)
-        got = to_bits(out)
+        out = self.torch.empty(token_major(q).shape, dtype=self.torch.bfloat16, device="cuda")
+        self.cache.temporal(layer, to_dev(token_major(q)), to_dev(token_major(k)), to_dev(token_major(v)), out, n)
+        got = np.ascontiguousarray(np.swapaxes(to_bits(out), 1, 2))
         pk, pv = self.rings[layer].prefix()
         if units is None:
             ref = oracle.temporal_attn(q, k, v, pk, pv)
@@ -104,7 +110,7 @@ class Loop:
     def write(self, kts, vts, kss, vss):
         n = kts[0].shape[1]
         e = self.cache.evict_for(n)
-        self.cache.write([to_dev(x) for x in kts], [to_dev(x) for x in vts],
+        self.cache.write([to_dev(token_major(x)) for x in kts], [to_dev(token_major(x)) for x in vts],
                          [to_dev(x) for x in kss], [to_dev(x) for x in vss], n)
         for L in range(self.wl.n_layers):
             gone = self.rings[L].write(kts[L], vts[L], kss[L], vss[L])
@@ -121,8 +127,8 @@ class Loop:
             rv = to_bits(self.cache.ring(L, 1))
             for g in ring.queue:
                 slot = ring.slot_of(g)
-                assert np.array_equal(rk[slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
-                assert np.array_equal(rv[slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rk[:, :, slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rv[:, :, slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
             if self.wl.p_spatial:
                 sk = to_bits(self.cache.spatial(L, 0))
                 sv = to_bits(self.cache.spatial(L, 1))

@@ -44,15 +44,16 @@ def test_first_frame_temporal_returns_v_exactly():
     1, so the output is V bit for bit."""
     import torch
     from causal_kv_cache_b200.ca2 import KVCache
-    from tests.gpu_util import to_bits, to_dev
+    from tests.gpu_util import to_bits, to_dev, token_major
     for name in ("tiny", "os_p41"):
         wl = WORKLOADS[name]
         g = Generator(wl, 3)
         q, k, v = g.qkv(1)
         c = KVCache(1, wl.batch, wl.hw, wl.heads, wl.head_dim, wl.chunk_len, wl.p_max, wl.p_spatial)
-        out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
-        c.temporal(0, to_dev(q), to_dev(k), to_dev(v), out, 1)
-        assert np.array_equal(to_bits(out), v)
+        tq, tk, tv = token_major(q), token_major(k), token_major(v)
+        out = torch.empty(tq.shape, dtype=torch.bfloat16, device="cuda")
+        c.temporal(0, to_dev(tq), to_dev(tk), to_dev(tv), out, 1)
+        assert np.array_equal(to_bits(out), tv)
 
 
 def test_os_p41_eighty_frames():
@@ -103,7 +104,7 @@ def test_cache_shared_across_denoising_steps_bit_identical():
     """Cache sharing: T reads of one cache give bit-identical outputs, the cache bytes do
     not change, and a cache rebuilt before each step gives the same bits again."""
     import torch
-    from tests.gpu_util import Loop, to_bits, to_dev
+    from tests.gpu_util import Loop, to_bits, to_dev, token_major
     wl = _wl("os_p41")
     lp = Loop(wl, seed=4)
     lp.first_frame()
@@ -111,7 +112,7 @@ def test_cache_shared_across_denoising_steps_bit_identical():
     lp.ar_step(wl.chunk_len, 0, s_units=np.arange(2))
     ring_before = lp.cache.tbuf.clone()
     sp_before = lp.cache.sbuf.clone()
-    tq, tk, tv = (to_dev(x) for x in lp.gen.qkv(wl.chunk_len))
+    tq, tk, tv = (to_dev(token_major(x)) for x in lp.gen.qkv(wl.chunk_len))
     sq, sk, sv = (to_dev(x) for x in lp.gen.qkv(wl.chunk_len))
     to = torch.empty_like(tq)
     so = torch.empty_like(sq)
@@ -144,7 +145,7 @@ def test_cache_shared_across_denoising_steps_bit_identical():
                 vs[:, hi - lo - len(ring.spatial_ids) + j] = ring.sv[g]
         else:
             ks, vs = kt, vt
-        c2.write([to_dev(kt)], [to_dev(vt)], [to_dev(ks)], [to_dev(vs)], hi - lo)
+        c2.write([to_dev(token_major(kt))], [to_dev(token_major(vt))], [to_dev(ks)], [to_dev(vs)], hi - lo)
     assert frames == list(range(17))
     to2 = torch.empty_like(tq)
     so2 = torch.empty_like(sq)
