@@ -322,7 +322,7 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     p.D = g.head_dim;
     p.n_src = 1 + n_sp;
     p.nkb = (g.hw + 127) / 128;
-    p.q_tiles = (g.hw + 127) / 128;
+    p.q_pairs = (g.hw + 255) / 256;
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
     return cuda_status(ca2::launch_spatial(m, p, static_cast<cudaStream_t>(stream)));
 }

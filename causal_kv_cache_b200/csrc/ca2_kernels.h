@@ -66,7 +66,7 @@ struct SpatialParams {
     int B, n, H, HW, D;
     int n_src;      // key sources: own frame + spatial-cache frames
     int nkb;        // 128-key blocks per source: ceil(HW / 128)
-    int q_tiles;    // 128-query tiles per frame: ceil(HW / 128)
+    int q_pairs;    // pairs of 128-query tiles per frame: ceil(HW / 256)
     float scale_log2;
 };
 
