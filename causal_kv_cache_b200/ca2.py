@@ -20,6 +20,7 @@ __all__ = [
     "ca2_cache_bytes", "ca2_cache_init", "ca2_cache_destroy", "ca2_cache_evict",
     "ca2_cache_write", "ca2_temporal_attn", "ca2_spatial_prefix_attn", "ca2_tpe_indices",
     "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string",
+    "ca2_last_error_string",
     "KVCache", "STATUS",
 ]
 
@@ -34,7 +35,13 @@ STATUS = {
 class Ca2Error(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__("%s failed: %s (%s)" % (where, STATUS.get(status, status), _string(status)))
+        detail = _string(status)
+        if status == -5:
+            try:
+                detail += ": " + load_library().ca2_last_error_string().decode()
+            except Exception:  # pragma: no cover
+                pass
+        super().__init__("%s failed: %s (%s)" % (where, STATUS.get(status, status), detail))
 
 
 class ca2_config(ctypes.Structure):
@@ -76,6 +83,7 @@ def load_library(path: Optional[str] = None):
         "ca2_device_status": ([], i),
         "ca2_selftest_timeout": ([i, vp], i),
         "ca2_status_string": ([i], ctypes.c_char_p),
+        "ca2_last_error_string": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -210,6 +218,10 @@ def ca2_selftest_timeout(wait_us: int, stream=None) -> None:
 
 def ca2_status_string(status: int) -> str:
     return load_library().ca2_status_string(int(status)).decode()
+
+
+def ca2_last_error_string() -> str:
+    return load_library().ca2_last_error_string().decode()
 
 
 # ---- convenience owner ------------------------------------------------------------------

@@ -51,7 +51,15 @@ size_t plane_bytes_of(const ca2_config *c)
     return (size_t)c->batch * (size_t)c->hw * (size_t)c->heads * (size_t)c->head_dim * 2u;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? CA2_OK : CA2_ERR_CUDA; }
+// Name of the last CUDA error a call of this library met (per host thread).
+thread_local const char *g_last_cuda_error = "no error";
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return CA2_OK;
+    g_last_cuda_error = cudaGetErrorString(e);
+    return CA2_ERR_CUDA;
+}
 
 int sm_count()
 {
@@ -230,8 +238,8 @@ int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t
             p.layer[i].ks = n_sp > 0 ? static_cast<const uint4 *>(k_s[L0 + i]) : nullptr;
             p.layer[i].vs = n_sp > 0 ? static_cast<const uint4 *>(v_s[L0 + i]) : nullptr;
         }
-        cudaError_t e = ca2::launch_cache_write(p, static_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return CA2_ERR_CUDA;
+        const int st = cuda_status(ca2::launch_cache_write(p, static_cast<cudaStream_t>(stream)));
+        if (st != CA2_OK) return st;
     }
     c->count += n;
     c->sp_count = n_sp;
@@ -274,7 +282,10 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
                   (long long)g.hw * g.p_max * C, 16, G) &&
         encode_5d(&m.rv, layer_ring(c, layer, 1), g.head_dim, g.p_max, g.heads, g.hw, g.batch, C, g.p_max * C,
                   (long long)g.hw * g.p_max * C, 16, G);
-    if (!ok) return CA2_ERR_CUDA;
+    if (!ok) {
+        g_last_cuda_error = "tensor-map encoding failed";
+        return CA2_ERR_CUDA;
+    }
     const int sms = sm_count();
     if (sms <= 0) return CA2_ERR_CUDA;
     int grid = 2 * sms;
@@ -293,27 +304,22 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     const int frames = g.batch * n;
     ca2::SpatialMaps m;
     const int D = g.head_dim, H = g.heads, HW = g.hw;
-    // wide boxes exist only when D >= 64; otherwise slot [0] is a copy that is never read
-    auto pair = [&](CUtensorMap *mm, const void *base, int frames_) {
-        if (!encode_4d(&mm[1], base, D, H, HW, frames_, 16, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
-        if (D < 64) {
-            mm[0] = mm[1];
-            return true;
-        }
-        return encode_4d(&mm[0], base, D, H, HW, frames_, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    auto load_map = [&](CUtensorMap *mm, const void *base, int frames_) {
+        return encode_4d(mm, base, D, H, HW, frames_, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
     };
-    bool ok = pair(m.q, q, frames) && pair(m.k, k, frames) && pair(m.v, v, frames) &&
+    bool ok = load_map(&m.q, q, frames) && load_map(&m.k, k, frames) && load_map(&m.v, v, frames) &&
               encode_4d(&m.o, out, D, H, HW, frames, D, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && n_sp > 0) {
-        ok = pair(m.sk, layer_spatial(c, layer, 0), n_sp * g.batch) &&
-             pair(m.sv, layer_spatial(c, layer, 1), n_sp * g.batch);
+        ok = load_map(&m.sk, layer_spatial(c, layer, 0), n_sp * g.batch) &&
+             load_map(&m.sv, layer_spatial(c, layer, 1), n_sp * g.batch);
     } else if (ok) {
-        for (int i = 0; i < 2; ++i) {   // never read when there is no prefix
-            m.sk[i] = m.k[i];
-            m.sv[i] = m.v[i];
-        }
+        m.sk = m.k;   // never read when there is no prefix
+        m.sv = m.v;
     }
-    if (!ok) return CA2_ERR_CUDA;
+    if (!ok) {
+        g_last_cuda_error = "tensor-map encoding failed";
+        return CA2_ERR_CUDA;
+    }
     ca2::SpatialParams p;
     p.B = g.batch;
     p.n = n;
@@ -361,6 +367,8 @@ int ca2_selftest_timeout(int wait_us, void *stream)
     return cuda_status(
         ca2::launch_timeout_selftest((unsigned long long)wait_us * 1000ull, static_cast<cudaStream_t>(stream)));
 }
+
+const char *ca2_last_error_string(void) { return g_last_cuda_error; }
 
 const char *ca2_status_string(int s)
 {

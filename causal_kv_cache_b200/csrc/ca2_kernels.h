@@ -70,10 +70,10 @@ struct SpatialParams {
     float scale_log2;
 };
 
-// Loaded tensors have two maps each: [0] boxes of 64 head-dims x 128 tokens (128-byte
-// swizzle), [1] boxes of 16 head-dims x 128 tokens (32-byte swizzle).  o: D x 128 tokens.
+// Loaded tensors: boxes of 32 head-dims x 128 tokens with the 64-byte swizzle.
+// o: boxes of D x 128 tokens, no swizzle (the output tile is staged dense in shared memory).
 struct SpatialMaps {
-    CUtensorMap q[2], k[2], v[2], sk[2], sv[2], o;
+    CUtensorMap q, k, v, sk, sv, o;
 };
 
 uint32_t spatial_smem_bytes(int D);

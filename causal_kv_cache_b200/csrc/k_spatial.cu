@@ -7,25 +7,29 @@
 // attention unchanged, so that mode reads the own frame once (n_src = 1).
 //
 // One CTA computes two 128-query tiles (A and B) of one (video, frame, head); each K/V
-// block is loaded once and used by both tiles.  Twelve warps:
-//   warp 0       TMA producer: both Q tiles, then K and V blocks of 128 keys into two
-//                independent rings (K is released as soon as both QK^T products have read
-//                it, V after both P V products).  An operand tile is one 64-column box per
-//                full 64 head-dims (128-byte rows, 128-byte swizzle) plus 16-column boxes
-//                for the rest (32-byte rows, 32-byte swizzle); columns past D (72 -> 80)
-//                and rows past HW are zero-filled by the TMA unit.
+// block is loaded once and used by both tiles.  Eighteen warps:
+//   warp 0       TMA producer (one thread): both Q tiles, then K and V blocks of 128
+//                keys into two independent rings (K is released as soon as both QK^T
+//                products have read it, V after both P V products).  An operand tile is
+//                ceil(D/32) boxes of 32 head-dims x 128 tokens (64-byte rows, 64-byte
+//                swizzle); columns past D (72 -> 96) and rows past HW are zero-filled by
+//                the TMA unit.  One block behind its loads the same thread prepares each
+//                landed V tile: when D is not a multiple of 32, padding column D is set to
+//                1.0, so the P V product also accumulates the row sum of the
+//                probabilities into O[:, D] (rescaled together with O).
 //   warp 1       MMA issuer (one thread) and TMEM owner (512 columns: S/P of A and B,
 //                then O of A and B).  Order per block j: P_A V, S_A(j+1), P_B V, S_B(j+1),
 //                so one tile's softmax always overlaps the other tile's products.
-//   warp 2       prepares each landed V block: when D is not a multiple of 16, padding
-//                column D is set to 1.0, so the P V product also accumulates the row sum
-//                of the probabilities into O[:, D] (rescaled together with O).
-//   warps 4-7    softmax of tile A, warps 8-11 softmax of tile B, one thread per query
-//                row (TMEM lane).  Pass 1 reads the 128 scores for the row max; the
-//                running max moves only when it grows by more than 2^8 (O is then
-//                rescaled in TMEM).  Pass 2 re-reads the scores 32 at a time, exponentiates
-//                and writes the bf16 probabilities back over the scores in TMEM, where the
-//                P V product reads them as its A operand.  Epilogue: O / l -> bf16 ->
+//   warps 2-17   softmax: 8 warps per tile, two threads per query row (TMEM lane; warp % 4
+//                selects the lane quarter), each taking 64 of a block's 128 keys; the two
+//                swap partial row maxima through shared memory.  The two tiles take turns
+//                on the exponential unit (measured 16 lanes/clock/SM, the scarce pipe), so
+//                one tile exponentiates while the other's products run.  The running max moves only
+//                when it grows by more than 2^8 (O is then rescaled in TMEM).  (Moving part
+//                of the exponentials to an FMA-pipe polynomial was measured slower: the
+//                warps are issue- and latency-bound, not bound by the exponential unit.)
+//                The bf16 probabilities are written back over the scores in TMEM, where
+//                the P V product reads them as its A operand.  Epilogue: O / l -> bf16 ->
 //                shared memory -> one TMA store per tile.
 //
 // Every mbarrier wait is bounded; a timeout is recorded in the library status word and
@@ -41,11 +45,11 @@ namespace ca2 {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 576;        // 18 warps
 constexpr int kRows = 128;           // queries per tile = TMEM lanes
 constexpr int kKeys = 128;           // keys per block
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSw128 = 2, kSw32 = 6;   // smem-descriptor layout codes
+constexpr uint32_t kSw64 = 4;               // smem-descriptor layout code: 64-byte swizzle
 constexpr float kLazyRescale = 8.0f;        // log2 units
 
 // ---- tcgen05 helpers ---------------------------------------------------------------------
@@ -176,26 +180,46 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// Two non-negative fp32 values -> packed bf16x2 (lo in the low half), rounded to nearest
-// (ties away from zero) with integer arithmetic: add half a bf16 ulp to the fp32 bits and
-// keep the high halves.  Keeps the conversion off the transcendental/conversion pipe.
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi)
+// 32 lanes x 128 consecutive 32-bit columns (two x64 loads, one wait).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
 {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(__float_as_uint(lo) + 0x8000u), "r"(__float_as_uint(hi) + 0x8000u));
-    return r;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+          "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+          "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+          "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+          "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+          "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]),
+          "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+          "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]),
+          "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+        : "r"(taddr), "r"(taddr + 64u)
+        : "memory");
 }
 
-// One operand tile (128 rows x padded D) is NA boxes of 64 columns with 128-byte rows and
-// the 128-byte swizzle (16 KB each), then NR boxes of 16 columns with 32-byte rows and the
-// 32-byte swizzle (4 KB each): NA = NKD / 4, NR = NKD % 4 for NKD = ceil(D / 16).
-__host__ __device__ constexpr uint32_t tile_bytes(int nkd) { return (nkd / 4) * 16384u + (nkd % 4) * 4096u; }
+// One operand tile (128 rows x padded D) is NB32 = ceil(D / 32) boxes of 32 columns with
+// 64-byte rows and the 64-byte swizzle (8 KB each).  64-byte rows stream at full speed
+// through the TMA unit, and one layout serves both products: K-major for Q and K (a
+// 16-column k-step is half a swizzled row) and MN-major for V, so P V is a single MMA of
+// N = 32 * NB32 per 16 keys.  Columns past D (72 -> 96) read as zero.
+__host__ __device__ constexpr int n32(int nkd) { return (nkd + 1) / 2; }
+__host__ __device__ constexpr uint32_t tile_bytes(int nkd) { return n32(nkd) * 8192u; }
 __host__ __device__ constexpr uint32_t tile_slot(int nkd) { return (tile_bytes(nkd) + 1023u) & ~1023u; }
 // K and V ring depth: three blocks when it fits in shared memory, else two
 __host__ __device__ constexpr int kv_stages(int nkd) { return 8 * tile_slot(nkd) + 1280u <= 232448u ? 3 : 2; }
 
 struct SmemLayout {
-    uint32_t q0, k0, v0, bars, total;
+    uint32_t q0, k0, v0, bars, red, total;
 };
 
 __host__ __device__ constexpr SmemLayout spatial_layout(int nkd)
@@ -205,7 +229,8 @@ __host__ __device__ constexpr SmemLayout spatial_layout(int nkd)
     L.k0 = 2 * tile_slot(nkd);
     L.v0 = L.k0 + kv_stages(nkd) * tile_slot(nkd);
     L.bars = L.v0 + kv_stages(nkd) * tile_slot(nkd);
-    L.total = L.bars + 256 + 1024;   // barriers + slack for the 1024-byte base alignment
+    L.red = L.bars + 512;            // row-max exchange: [2][2][2][128] floats
+    L.total = L.red + 4096 + 1024;   // + slack for the 1024-byte base alignment
     return L;
 }
 
@@ -220,21 +245,23 @@ enum : int {
     B_SFULL = 16,     // 2 (tile A, B): scores in TMEM (implies the previous P V done)
     B_PFULL = 18,     // 2: probabilities in TMEM (4 softmax warps)
     B_ODONE = 20,     // 2: P V of the tile done
-    B_OSTAGED = 22,   // 2: output rows of the tile in shared memory (4 warps)
-    B_COUNT = 24
+    B_OSTAGED = 22,   // 2: output rows of the tile in shared memory (8 warps)
+    B_XCH = 24,       // 8 (tile x lane quarter): partial row maxima of both halves written
+    B_EXP = 32,       // 2: a tile's exponential phase of a block is over (8 warps)
+    B_COUNT = 34
 };
 
 }  // namespace
 
 template <int NKD>
 __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_constant__ SpatialMaps tm,
-                                                                  const SpatialParams p)
+                                                   const SpatialParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     constexpr SmemLayout L = spatial_layout(NKD);
     constexpr int NS = kv_stages(NKD);
-    constexpr int NA = NKD / 4;                  // 64-column boxes (128-byte swizzle)
-    constexpr int NR = NKD % 4;                  // 16-column boxes (32-byte swizzle)
+    constexpr int NB32 = n32(NKD);               // 32-column boxes per operand tile
+    constexpr int DP = 32 * NB32;                // P V width (padded head dim)
     constexpr uint32_t TB = tile_slot(NKD);
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;  // 1024-aligned base for the swizzled tiles
@@ -270,21 +297,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(B_SFULL + i), 1);
-            mbar_init(bar(B_PFULL + i), 4);
+            mbar_init(bar(B_PFULL + i), 8);
             mbar_init(bar(B_ODONE + i), 1);
-            mbar_init(bar(B_OSTAGED + i), 4);
+            mbar_init(bar(B_OSTAGED + i), 8);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(bar(B_XCH + i), 2);
+        for (int i = 0; i < 2; ++i) mbar_init(bar(B_EXP + i), 8);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        for (int i = 0; i < 2; ++i) {
-            prefetch_tmap(&tm.q[i]);
-            prefetch_tmap(&tm.k[i]);
-            prefetch_tmap(&tm.v[i]);
-            prefetch_tmap(&tm.sk[i]);
-            prefetch_tmap(&tm.sv[i]);
-        }
+        prefetch_tmap(&tm.q);
+        prefetch_tmap(&tm.k);
+        prefetch_tmap(&tm.v);
+        prefetch_tmap(&tm.sk);
+        prefetch_tmap(&tm.sv);
         prefetch_tmap(&tm.o);
     }
     if (warp == 1) {
@@ -295,41 +322,63 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // When D is not a multiple of 16 the P V product has padding columns D..DP-1; column D
+    // When D is not a multiple of 32 the P V product has padding columns D..DP-1; column D
     // of every V tile is set to 1.0 so that the tensor core also accumulates the row sum
     // of the (bf16) probabilities into O[:, D], rescaled together with O.
-    const bool ones_col = (p.D & 15) != 0;
+    const bool ones_col = (p.D & 31) != 0;
 
     if (warp == 0) {
         // ------------------------------- TMA producer (one thread) --------------------
         if (lane == 0) {
-            // one operand tile: NA wide boxes then NR narrow boxes
-            auto load_tile = [&](uint32_t dst, const CUtensorMap *maps, int r0, int fr, uint32_t bar_addr) {
-                for (int a = 0; a < NA; ++a) tma_load_4d(dst + a * 16384u, &maps[0], 64 * a, h, r0, fr, bar_addr);
-                for (int r = 0; r < NR; ++r)
-                    tma_load_4d(dst + NA * 16384u + r * 4096u, &maps[1], 64 * NA + 16 * r, h, r0, fr, bar_addr);
+            // one operand tile: NB32 boxes of 32 columns
+            auto load_tile = [&](uint32_t dst, const CUtensorMap *map, int r0, int fr, uint32_t bar_addr) {
+                for (int a = 0; a < NB32; ++a) tma_load_4d(dst + a * 8192u, map, 32 * a, h, r0, fr, bar_addr);
             };
             mbar_expect_tx(bar(B_QFULL), 2 * tile_bytes(NKD));
-            load_tile(sb + L.q0, tm.q, row0, b * p.n + f, bar(B_QFULL));
-            load_tile(sb + L.q0 + TB, tm.q, row0 + kRows, b * p.n + f, bar(B_QFULL));
+            load_tile(sb + L.q0, &tm.q, row0, b * p.n + f, bar(B_QFULL));
+            load_tile(sb + L.q0 + TB, &tm.q, row0 + kRows, b * p.n + f, bar(B_QFULL));
+            // V preparation (one block behind the issue): when D is not a multiple of 32,
+            // column D of the landed V tile := 1.0 (bf16 0x3F80) at its swizzled address
+            // (64-byte rows, 16-byte chunk index ^= (row >> 1) & 3); then V is ready
+            auto prep = [&](int jv) -> bool {
+                const int s = jv % NS;
+                if (!mbar_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
+                if (ones_col) {
+                    const uint32_t vt = sb + L.v0 + s * TB;
+                    const int D = p.D;
+                    const int c = (D & 31) >> 3;
+                    const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
+#pragma unroll 4
+                    for (int r = 0; r < kKeys; ++r)
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
+                                     "h"((unsigned short)0x3F80)
+                                     : "memory");
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(bar(B_VREADY + s));
+                return true;
+            };
             int issued_k = -1, issued_v = -1;
-            for (int j = 0; j < NB; ++j) {
+            bool ok = true;
+            for (int j = 0; ok && j < NB; ++j) {
                 const int s = j % NS;
                 const int u = j / NS;
                 const int src = j / p.nkb;
                 const int kb = j - src * p.nkb;
-                const CUtensorMap *mk = src == 0 ? tm.k : tm.sk;
-                const CUtensorMap *mv = src == 0 ? tm.v : tm.sv;
+                const CUtensorMap *mk = src == 0 ? &tm.k : &tm.sk;
+                const CUtensorMap *mv = src == 0 ? &tm.v : &tm.sv;
                 const int fr = src == 0 ? b * p.n + f : (src - 1) * p.B + b;
-                if (j >= NS && !mbar_wait(bar(B_KEMPTY + s), (u - 1) & 1, 201, abort_flag)) break;
+                if (j >= NS && !mbar_wait(bar(B_KEMPTY + s), (u - 1) & 1, 201, abort_flag)) { ok = false; break; }
                 mbar_expect_tx(bar(B_KFULL + s), tile_bytes(NKD));
                 load_tile(sb + L.k0 + s * TB, mk, kb * kKeys, fr, bar(B_KFULL + s));
                 issued_k = j;
-                if (j >= NS && !mbar_wait(bar(B_VEMPTY + s), (u - 1) & 1, 202, abort_flag)) break;
+                if (j >= NS && !mbar_wait(bar(B_VEMPTY + s), (u - 1) & 1, 202, abort_flag)) { ok = false; break; }
                 mbar_expect_tx(bar(B_VFULL + s), tile_bytes(NKD));
                 load_tile(sb + L.v0 + s * TB, mv, kb * kKeys, fr, bar(B_VFULL + s));
                 issued_v = j;
+                if (j >= 1 && !prep(j - 1)) ok = false;
             }
+            if (ok && NB > 0) prep(NB - 1);
             // wind-down after an abort: let every issued load land before the CTA exits
             // (each ring slot's last use is the most recent phase of its barrier)
             if (*abort_flag) {
@@ -340,67 +389,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                     mbar_wait(bar(B_VFULL + j % NS), (j / NS) & 1, 0, nullptr, 2000000ull);
             }
         }
-    } else if (warp == 2) {
-        // ------------------------------- V preparation ---------------------------------
-        for (int j = 0; j < NB; ++j) {
-            const int s = j % NS;
-            if (!warp_wait(bar(B_VFULL + s), (j / NS) & 1, 203, abort_flag)) break;
-            if (ones_col) {
-                // column D of this V tile := 1.0 (bf16 0x3F80), at its swizzled address
-                const uint32_t vt = sb + L.v0 + s * TB;
-                const int D = p.D;
-                for (int r = lane; r < kKeys; r += 32) {
-                    uint32_t a;
-                    if (D < 64 * NA) {          // inside a 64-column box: 128-byte rows, 128-byte swizzle
-                        const int c = (D & 63) >> 3;
-                        a = vt + (uint32_t)(D >> 6) * 16384u + (uint32_t)r * 128u +
-                            (uint32_t)(((c ^ (r & 7)) << 4) + (D & 7) * 2);
-                    } else {                    // inside a 16-column box: 32-byte rows, 32-byte swizzle
-                        const int e = D - 64 * NA;
-                        a = vt + (uint32_t)NA * 16384u + (uint32_t)(e >> 4) * 4096u + (uint32_t)r * 32u +
-                            (uint32_t)(((((e & 15) >> 3) ^ ((r >> 2) & 1)) << 4) + (e & 7) * 2);
-                    }
-                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((unsigned short)0x3F80) : "memory");
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_VREADY + s));
-        }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer (one thread) -----------------------
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
-            constexpr uint32_t idesc_pv_w = idesc_bf16(kRows, NA > 0 ? 64 * NA : 16, false, true);
-            constexpr uint32_t idesc_pv_n = idesc_bf16(kRows, NR > 0 ? 16 * NR : 16, false, true);
-            // K-major operand descriptor of k-step kk inside a tile at `tile`
-            auto kdesc = [&](uint32_t tile, int kk) -> uint64_t {
-                if (kk < 4 * NA) return sdesc(tile + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024, kSw128);
-                return sdesc(tile + NA * 16384u + (kk - 4 * NA) * 4096u, 16, 256, kSw32);
-            };
+            constexpr uint32_t idesc_pv = idesc_bf16(kRows, DP, false, true);
+            // Descriptors are built once; a k-step only adds its byte offset / 16 to the
+            // start-address field (addresses stay below 256 KB, so no carry leaves it).
+            // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
+            // MN-major (V): atoms of 32 head-dims 8 KB apart (LBO), 8-key groups 512 B apart.
+            // (stage tiles are TB bytes apart, so one base descriptor per ring suffices)
+            const uint64_t dq0 = sdesc(sb + L.q0, 16, 512, kSw64);
+            const uint64_t dk0 = sdesc(sb + L.k0, 16, 512, kSw64);
+            const uint64_t dv0 = sdesc(sb + L.v0, 8192, 512, kSw64);
+            auto koff = [](int kk) -> uint64_t { return (uint64_t)(((kk >> 1) * 8192 + (kk & 1) * 32) >> 4); };
             // S_X = Q_X K^T into TMEM columns [128 X, 128 X + 128)
             auto issue_qk = [&](int X, int j) {
-                const uint32_t kt = sb + L.k0 + (j % NS) * TB;
-                const uint32_t qt = sb + L.q0 + X * TB;
+                const uint64_t bk = dk0 + (uint64_t)(((j % NS) * TB) >> 4), bq = dq0 + (uint64_t)((X * TB) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < NKD; ++kk)
-                    tc_mma_ss(tmem + X * kKeys, kdesc(qt, kk), kdesc(kt, kk), idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(tmem + X * kKeys, bq + koff(kk), bk + koff(kk), idesc_qk, kk > 0 ? 1u : 0u);
                 tc_commit(bar(B_SFULL + X));
             };
-            // O_X (+)= P_X V, P_X read from TMEM (two bf16 per column, 8 columns per 16 keys);
-            // V is MN-major: wide boxes of 64 dims (atoms 16 KB apart), narrow boxes of 16
+            // O_X (+)= P_X V, P_X read from TMEM (two bf16 per column, 8 columns per 16 keys)
             auto issue_pv = [&](int X, int j) {
-                const uint32_t vt = sb + L.v0 + (j % NS) * TB;
+                const uint64_t bv = dv0 + (uint64_t)(((j % NS) * TB) >> 4);
                 const uint32_t o = tmem + 2 * kKeys + X * kKeys;
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    const uint32_t a = tmem + X * kKeys + 8 * kk;
-                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                    if (NA > 0) tc_mma_ts(o, a, sdesc(vt + kk * 2048u, 16384, 1024, kSw128), idesc_pv_w, acc);
-                    if (NR > 0)
-                        tc_mma_ts(o + 64 * NA, a, sdesc(vt + NA * 16384u + kk * 512u, 4096, 256, kSw32), idesc_pv_n,
-                                  acc);
-                }
+                for (int kk = 0; kk < kKeys / 16; ++kk)
+                    tc_mma_ts(o, tmem + X * kKeys + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
+                              (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(B_ODONE + X));
             };
             int done_a = 0, done_b = 0;   // P V products issued per tile
@@ -441,44 +459,64 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             if (done_a > 0) mbar_wait(bar(B_ODONE + 0), (done_a - 1) & 1, 0, nullptr, 2000000ull);
             if (done_b > 0) mbar_wait(bar(B_ODONE + 1), (done_b - 1) & 1, 0, nullptr, 2000000ull);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         // ------------------------------- softmax / epilogue ---------------------------
-        const int X = (warp - 4) >> 2;                    // 0: tile A, 1: tile B
+        // 16 warps (2..17): tile X = sw / 8, half hh = (sw / 4) % 2 of a block's 128 keys,
+        // lane quarter = warp % 4 (each group of four consecutive warps covers all four).
+        // The two threads of a query row (same lane, warps sw and sw ^ 4) exchange their
+        // partial row maxima through shared memory once per block.
+        const int sw = warp - 2;
+        const int X = sw >> 3;
+        const int hh = (sw >> 2) & 1;
         const int quarter = warp & 3;                     // TMEM lanes 32*quarter ..
         const int row = quarter * 32 + lane;              // query row of this thread in its tile
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_col = tmem + lane_bits + X * kKeys;
         const uint32_t o_col = tmem + lane_bits + 2 * kKeys + X * kKeys;
+        const uint32_t xch = bar(B_XCH + X * 4 + quarter);
+        float *red = reinterpret_cast<float *>(sgen + L.red);   // [parity][tile][half][row]
+        auto red_at = [&](int par, int half) -> float & { return red[((par * 2 + X) * 2 + half) * kRows + row]; };
         const float neg_inf = __int_as_float(0xff800000);
         const float scale = p.scale_log2;
         float m_used = neg_inf;     // max (log2 units) the probabilities are taken against
-        float l_sum = 0.f;         // row sum, kept here only when there is no padding column
+        float l_sum = 0.f;         // partial row sum, kept only when there is no padding column
         bool ok = true;
+        int nx = 0;                 // exchanges done (phase counter of xch)
+        // exchange one float with the row's partner thread; false if the wait gave up
+        auto exchange = [&](float mine, float &theirs) -> bool {
+            red_at(nx & 1, hh) = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xch);
+            if (!warp_wait(xch, nx & 1, 226, abort_flag)) return false;
+            theirs = red_at(nx & 1, hh ^ 1);
+            ++nx;
+            return true;
+        };
         for (int j = 0; j < NB; ++j) {
             const int kb = j % p.nkb;
-            const int valid = min(kKeys, p.HW - kb * kKeys);
+            const int valid = min(kKeys, p.HW - kb * kKeys) - 64 * hh;   // valid keys of this half
             // S_X(j) ready; its commit also covers the previous P V of this tile
             if (!warp_wait(bar(B_SFULL + X), j & 1, 221, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            // pass 1: row max over the valid keys
+            // pass 1: this half's 64 scores into registers, partial row max, exchange
+            uint32_t sr[64];
+            tmem_ld64(s_col + 64 * hh, sr);
             float m8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = neg_inf;
+            if (valid >= 64) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[64];
-                tmem_ld64(s_col + 64 * half, r);
-                if (valid >= kKeys) {
+                for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(r[i]));
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (64 * half + i < valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(r[i]));
-                }
+                for (int i = 0; i < 64; ++i)
+                    if (i < valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
             }
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale;
+            const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            float qm;
+            if (!exchange(pm, qm)) { ok = false; break; }
+            const float mx = fmaxf(pm, qm) * scale;
             float alpha = 1.f;
             const bool upd = mx > m_used + kLazyRescale;
             if (upd) {
@@ -486,36 +524,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 m_used = mx;
             }
             if (j > 0 && __any_sync(0xffffffffu, upd)) {
+                // this thread's half of the row's O columns
 #pragma unroll
-                for (int c = 0; c < NKD; ++c) {
+                for (int c = 0; c < DP / 32; ++c) {
                     uint32_t o[16];
-                    tmem_ld16(o_col + 16 * c, o);
+                    const uint32_t a = o_col + (uint32_t)(hh * (DP / 2) + 16 * c);
+                    tmem_ld16(a, o);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st16(o_col + 16 * c, o);
+                    tmem_st16(a, o);
                 }
             }
             l_sum *= alpha;
-            // pass 2: probabilities, 32 keys at a time, written over the scores as bf16 pairs
+            // The two tiles take turns on the exponential unit (16 lanes/clock/SM, the
+            // scarce pipe): tile B's block j waits for tile A's block j, tile A's block
+            // j+1 for tile B's block j, so each tile's products run on the tensor core
+            // while the other tile exponentiates.
+            if (X == 1 || j > 0) {
+                const int other_j = X == 1 ? j : j - 1;
+                if (!warp_wait(bar(B_EXP + (X ^ 1)), other_j & 1, 227, abort_flag)) { ok = false; break; }
+            }
+            // pass 2: probabilities from the registers, written over the scores in TMEM as
+            // bf16 pairs (keys 64 hh + 32 c .. go to columns 32 hh + 16 c ..)
             const float neg_m = -m_used;
             float ls = 0.f;
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
-                uint32_t r[32], w[16];
-                tmem_ld32(s_col + 32 * c, r);
+            for (int c = 0; c < 2; ++c) {
+                uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float e0 = ex2(fmaf(__uint_as_float(r[2 * i]), scale, neg_m));
-                    float e1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), scale, neg_m));
-                    if (valid < kKeys) {
-                        if (32 * c + 2 * i >= valid) e0 = 0.f;
-                        if (32 * c + 2 * i + 1 >= valid) e1 = 0.f;
+                    const int k0 = 32 * c + 2 * i;
+                    float e0 = ex2(fmaf(__uint_as_float(sr[k0]), scale, neg_m));
+                    float e1 = ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale, neg_m));
+                    if (valid < 64) {
+                        if (k0 >= valid) e0 = 0.f;
+                        if (k0 + 1 >= valid) e1 = 0.f;
                     }
-                    w[i] = pack_bf16x2_pos(e0, e1);
+                    w[i] = pack_bf16x2(e0, e1);
                     if (!ones_col) ls += bf16_lo(w[i]) + bf16_hi(w[i]);
                 }
-                tmem_st16(s_col + 16 * c, w);
+                tmem_st16(s_col + (uint32_t)(32 * hh + 16 * c), w);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_EXP + X));
             l_sum += ls;
             tmem_st_wait();
             tc_fence_before();
@@ -532,39 +583,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     if (i == (p.D & 15)) l = __uint_as_float(o[i]);
+            } else {
+                float lt = 0.f;
+                if (!exchange(l_sum, lt)) ok = false;
+                l = l_sum + lt;
             }
             const float inv = 1.f / l;
             uint8_t *orow = sgen + L.q0 + X * TB + (size_t)row * (size_t)(p.D * 2);
 #pragma unroll
-            for (int c = 0; c < NKD; ++c) {
+            for (int c = 0; c < DP / 32; ++c) {
+                const int col = hh * (DP / 2) + 16 * c;   // first head-dim of this chunk
                 uint32_t o[16];
-                tmem_ld16(o_col + 16 * c, o);
+                tmem_ld16(o_col + (uint32_t)col, o);
 #pragma unroll
                 for (int hlf = 0; hlf < 2; ++hlf) {
-                    if (16 * c + 8 * hlf < p.D) {
-                        const float *v = reinterpret_cast<const float *>(o) + 8 * hlf;
+                    if (col + 8 * hlf < p.D) {
+                        auto v = [&](int i) { return __uint_as_float(o[8 * hlf + i]) * inv; };
                         uint4 w;
-                        w.x = pack_bf16x2(v[0] * inv, v[1] * inv);
-                        w.y = pack_bf16x2(v[2] * inv, v[3] * inv);
-                        w.z = pack_bf16x2(v[4] * inv, v[5] * inv);
-                        w.w = pack_bf16x2(v[6] * inv, v[7] * inv);
-                        *reinterpret_cast<uint4 *>(orow + 32 * c + 16 * hlf) = w;
+                        w.x = pack_bf16x2(v(0), v(1));
+                        w.y = pack_bf16x2(v(2), v(3));
+                        w.z = pack_bf16x2(v(4), v(5));
+                        w.w = pack_bf16x2(v(6), v(7));
+                        *reinterpret_cast<uint4 *>(orow + 2 * col + 16 * hlf) = w;
                     }
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_OSTAGED + X));
+            if (ok && lane == 0) mbar_arrive(bar(B_OSTAGED + X));
         }
         // tile rows entirely past HW are not stored
-        if (quarter == 0 && lane == 0 && row0 + X * kRows < p.HW &&
+        if (sw == 8 * X && lane == 0 && row0 + X * kRows < p.HW &&
             mbar_wait(bar(B_OSTAGED + X), 0, 225, abort_flag)) {
             tma_store_4d(&tm.o, sb + L.q0 + X * TB, 0, h, row0 + X * kRows, b * p.n + f);
             bulk_commit();
             bulk_wait_read<0>();
         }
     }
-
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

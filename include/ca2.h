@@ -158,6 +158,10 @@ int ca2_selftest_timeout(int wait_us, void *stream);
 /* Static description of an error code. */
 const char *ca2_status_string(int status);
 
+/* Text of the last CUDA error met by a call of this library on the calling host thread
+ * (the cause behind a CA2_ERR_CUDA), or "no error".  The string is static. */
+const char *ca2_last_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif
