@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ca2", choices=["ca2", "reference"])
     ap.add_argument("--layers", type=int, default=WORKLOAD["n_layers"])
@@ -196,42 +196,47 @@ def run_ca2(args):
     cap_sp = int(cap.cuda_stream)
     live_graphs = []
 
-    def direct_pass(use_prefix, ev):
-        for L in range(NL):
-            p = P[L]
-            if ev is not None:
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-                e0.record(stream)
-            spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, sp)
-            if ev is not None:
-                e1.record(stream)
-            tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, sp)
-            if ev is not None:
-                e2.record(stream)
-                ev.append(("den" if use_prefix else "self", e0, e1, e2))
-
-    def step(ev=None):
-        """One AR step: TPE indices, T denoising passes, the cache-writing pass, evict, write.
-
-        The queue state is fixed until the write, so the denoising pass (28 blocks x 2
-        kernels) is captured once into a CUDA graph and replayed; pass 0 and the
-        cache-writing pass are launched directly with CUDA events around every kernel."""
-        ca2.ca2_tpe_indices(h, g0[0], 0, l)
+    def capture(use_prefix, timed):
+        """One pass over the 28 blocks (spatial then temporal attention per block) captured
+        into a CUDA graph.  A timed capture brackets every kernel with event-record nodes,
+        so per-kernel device times come from the replay itself, with no host gaps."""
         graph = torch.cuda.CUDAGraph()
+        evs = []
         with torch.cuda.stream(cap):
             graph.capture_begin()
             for L in range(NL):
                 p = P[L]
-                spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, 1, cap_sp)
+                if timed:
+                    e0, e1, e2 = (torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
+                    e0.record(cap)
+                spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, cap_sp)
+                if timed:
+                    e1.record(cap)
                 tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, cap_sp)
+                if timed:
+                    e2.record(cap)
+                    evs.append(("den" if use_prefix else "self", e0, e1, e2))
             graph.capture_end()
         live_graphs.append(graph)
-        direct_pass(1, ev)
+        return graph, evs
+
+    def step(ev=None):
+        """One AR step: TPE indices, T denoising passes, the cache-writing pass, evict, write.
+
+        The queue state is fixed until the write, so each pass is a CUDA graph captured
+        once per step.  Pass 0 and the cache-writing pass replay timed graphs (event nodes
+        around every kernel); passes 1..T-1 replay the plain denoising graph."""
+        ca2.ca2_tpe_indices(h, g0[0], 0, l)
+        g_den, _ = capture(1, False)
+        g_den_t, e_den = capture(1, True)
+        g_self_t, e_self = capture(0, True)
+        g_den_t.replay()
         for t in range(1, T):
-            graph.replay()
-        direct_pass(0, ev)
+            g_den.replay()
+        g_self_t.replay()
         cache.evict_for(l)
         if ev is not None:
+            ev.extend(e_den + e_self)
             e3, e4 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
             e3.record(stream)
         ca2.ca2_cache_write(h, KT, VT, KS, VS, l, sp)

@@ -308,7 +308,7 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
         return encode_4d(mm, base, D, H, HW, frames_, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
     };
     bool ok = load_map(&m.q, q, frames) && load_map(&m.k, k, frames) && load_map(&m.v, v, frames) &&
-              encode_4d(&m.o, out, D, H, HW, frames, D, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+              encode_4d(&m.o, out, D, H, HW, frames, D, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && n_sp > 0) {
         ok = load_map(&m.sk, layer_spatial(c, layer, 0), n_sp * g.batch) &&
              load_map(&m.sv, layer_spatial(c, layer, 1), n_sp * g.batch);

@@ -71,7 +71,7 @@ struct SpatialParams {
 };
 
 // Loaded tensors: boxes of 32 head-dims x 128 tokens with the 64-byte swizzle.
-// o: boxes of D x 128 tokens, no swizzle (the output tile is staged dense in shared memory).
+// o: boxes of D x 32 tokens, no swizzle (each softmax warp stores its 32 output rows).
 struct SpatialMaps {
     CUtensorMap q, k, v, sk, sv, o;
 };

@@ -7,30 +7,32 @@
 // attention unchanged, so that mode reads the own frame once (n_src = 1).
 //
 // One CTA computes two 128-query tiles (A and B) of one (video, frame, head); each K/V
-// block is loaded once and used by both tiles.  Eighteen warps:
-//   warp 0       TMA producer (one thread): both Q tiles, then K and V blocks of 128
-//                keys into two independent rings (K is released as soon as both QK^T
-//                products have read it, V after both P V products).  An operand tile is
-//                ceil(D/32) boxes of 32 head-dims x 128 tokens (64-byte rows, 64-byte
-//                swizzle); columns past D (72 -> 96) and rows past HW are zero-filled by
-//                the TMA unit.  One block behind its loads the same thread prepares each
-//                landed V tile: when D is not a multiple of 32, padding column D is set to
-//                1.0, so the P V product also accumulates the row sum of the
-//                probabilities into O[:, D] (rescaled together with O).
-//   warp 1       MMA issuer (one thread) and TMEM owner (512 columns: S/P of A and B,
-//                then O of A and B).  Order per block j: P_A V, S_A(j+1), P_B V, S_B(j+1),
-//                so one tile's softmax always overlaps the other tile's products.
-//   warps 2-17   softmax: 8 warps per tile, two threads per query row (TMEM lane; warp % 4
-//                selects the lane quarter), each taking 64 of a block's 128 keys; the two
-//                swap partial row maxima through shared memory.  The two tiles take turns
-//                on the exponential unit (measured 16 lanes/clock/SM, the scarce pipe), so
-//                one tile exponentiates while the other's products run.  The running max moves only
-//                when it grows by more than 2^8 (O is then rescaled in TMEM).  (Moving part
-//                of the exponentials to an FMA-pipe polynomial was measured slower: the
-//                warps are issue- and latency-bound, not bound by the exponential unit.)
-//                The bf16 probabilities are written back over the scores in TMEM, where
-//                the P V product reads them as its A operand.  Epilogue: O / l -> bf16 ->
-//                shared memory -> one TMA store per tile.
+// block is loaded once and used by both tiles.  Twelve warps:
+//   warp 0       TMA producer: both Q tiles, then K and V blocks of 128 keys into two
+//                independent rings (K is released as soon as both QK^T products have read
+//                it, V after both P V products).  An operand tile is ceil(D/32) boxes of 32
+//                head-dims x 128 tokens (64-byte rows, 64-byte swizzle); columns past D
+//                (72 -> 96) and rows past HW are zero-filled by the TMA unit.  One block
+//                behind its loads the warp prepares each landed V tile: when D is not a
+//                multiple of 32, padding column D is set to 1.0, so the P V product also
+//                accumulates the row sum of the probabilities into O[:, D].
+//   warps 1, 2   MMA issuers of tile A and tile B (one thread each; warp 1 owns the 512
+//                TMEM columns).  A single thread issues about one tcgen05.mma per ~100
+//                cycles whatever the tile width, so each tile has its own issuer.  The
+//                tile's next QK^T is issued as soon as its softmax warps have read the
+//                current scores, and its P V product chunk by chunk as the probabilities
+//                land, so the tensor core works while the exponentials run.
+//   warp 3       idle.
+//   warps 4-11   softmax: 4 warps per tile, one thread per query row (its TMEM lane; warp
+//                % 4 selects the lane quarter) holding all 128 scores of a block in
+//                registers, so the row max needs no exchange.  The exponential unit
+//                (measured 16 lanes/clock/SM) is the scarce pipe.  The two tiles fill one
+//                shared TMEM probability region in turns, chunk by chunk, each turn
+//                waiting for the P V products of the previous one.  The running max moves
+//                only when it grows by more than 2^8 (O is then rescaled in TMEM).  The
+//                bf16 probabilities are the A operand of the P V product, read from TMEM.
+//                Epilogue: O / l -> bf16 rows staged in the tile's spent Q buffer -> one
+//                TMA store of 32 rows per warp.
 //
 // Every mbarrier wait is bounded; a timeout is recorded in the library status word and
 // all roles wind down through the common exit, which frees TMEM.
@@ -45,7 +47,7 @@ namespace ca2 {
 
 namespace {
 
-constexpr int kThreads = 576;        // 18 warps
+constexpr int kThreads = 384;        // 12 warps
 constexpr int kRows = 128;           // queries per tile = TMEM lanes
 constexpr int kKeys = 128;           // keys per block
 constexpr uint32_t kTmemCols = 512;
@@ -234,22 +236,46 @@ __host__ __device__ constexpr SmemLayout spatial_layout(int nkd)
     return L;
 }
 
-// barrier indices (K/V rings have up to three stages)
+// TMEM columns (512 allocated).  When the padded head dim DP is at most 96 the two tiles
+// keep separate score regions and share one probability region:
+//   S_A [0,128)  S_B [128,256)  P [256,320)  O_A [320,320+DP)  O_B [320+DP,320+2DP)
+// so a tile's next scores can be computed while its probabilities are still being
+// written and read.  With DP = 128 there is no room for that: P is written over the
+// tile's own scores and the next QK^T waits for the P V product.
+template <int NB32>
+struct TmemMap {
+    static constexpr int DP = 32 * NB32;
+    static constexpr bool kSharedP = NB32 <= 3;
+    __host__ __device__ static constexpr uint32_t s(int X) { return (uint32_t)X * 128u; }
+    __host__ __device__ static constexpr uint32_t p(int X) { return kSharedP ? 256u : (uint32_t)X * 128u; }
+    __host__ __device__ static constexpr uint32_t o(int X)
+    {
+        return kSharedP ? 320u + (uint32_t)(X * DP) : 256u + (uint32_t)X * 128u;
+    }
+};
+static_assert(TmemMap<3>::o(1) + 96 <= kTmemCols, "TMEM map overflows");
+static_assert(TmemMap<4>::o(1) + 128 <= kTmemCols, "TMEM map overflows");
+
+constexpr int kChunks = 4;            // probability chunks per block: 32 keys = 16 P columns each
+constexpr int kSoftmaxWarp0 = 4;      // warps 4..7 tile A, 8..11 tile B
+
+// barrier indices (K/V rings have up to three stages; X = tile, c = probability chunk)
 enum : int {
     B_QFULL = 0,
     B_KFULL = 1,      // 3
-    B_KEMPTY = 4,     // 3: both QK^T products of the block are done
+    B_KEMPTY = 4,     // 3: both tiles' QK^T of the block are done (2 commits)
     B_VFULL = 7,      // 3
     B_VREADY = 10,    // 3: padding column prepared
-    B_VEMPTY = 13,    // 3: both P V products of the block are done
-    B_SFULL = 16,     // 2 (tile A, B): scores in TMEM (implies the previous P V done)
-    B_PFULL = 18,     // 2: probabilities in TMEM (4 softmax warps)
-    B_ODONE = 20,     // 2: P V of the tile done
-    B_OSTAGED = 22,   // 2: output rows of the tile in shared memory (8 warps)
-    B_XCH = 24,       // 8 (tile x lane quarter): partial row maxima of both halves written
-    B_EXP = 32,       // 2: a tile's exponential phase of a block is over (8 warps)
-    B_COUNT = 34
+    B_VEMPTY = 13,    // 3: both tiles' P V of the block are done (2 commits)
+    B_SFULL = 16,     // 2 [X]: scores in TMEM
+    B_SFREE = 18,     // 2 [X]: every softmax warp of the tile has read the scores (4 warps)
+    B_PFULL = 20,     // 8 [X][c]: probability chunk in TMEM (4 warps)
+    B_PFREE = 28,     // 4 [c]: the P V products reading the shared chunk are done
+    B_ODONE = 32,     // 2 [X]: P V of the block done (all prior products of the tile)
+    B_FIN = 34,       // 2 [X]: every product the tile's issuer launched is done
+    B_COUNT = 36
 };
+static_assert(8 * B_COUNT + 12 <= 512, "barrier area");
 
 }  // namespace
 
@@ -263,6 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     constexpr int NB32 = n32(NKD);               // 32-column boxes per operand tile
     constexpr int DP = 32 * NB32;                // P V width (padded head dim)
     constexpr uint32_t TB = tile_slot(NKD);
+    using TM = TmemMap<NB32>;
+    constexpr bool kSharedP = TM::kSharedP;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;  // 1024-aligned base for the swizzled tiles
     uint8_t *sgen = smem_raw + (sb - raw);
@@ -286,33 +314,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     const int NB = p.n_src * p.nkb;
     const int row0 = qp * 2 * kRows;             // first query row of tile A; tile B follows
 
+    // one operand tile: NB32 boxes of 32 columns
+    auto load_tile = [&](uint32_t dst, const CUtensorMap *map, int r0, int fr, uint32_t bar_addr) {
+        for (int a = 0; a < NB32; ++a) tma_load_4d(dst + a * 8192u, map, 32 * a, h, r0, fr, bar_addr);
+    };
+    // key block j -> (tensor map, first key row, frame index)
+    auto kv_src = [&](int j, const CUtensorMap *&mk, const CUtensorMap *&mv, int &r, int &fr) {
+        const int src = j / p.nkb;
+        r = (j - src * p.nkb) * kKeys;
+        mk = src == 0 ? &tm.k : &tm.sk;
+        mv = src == 0 ? &tm.v : &tm.sv;
+        fr = src == 0 ? b * p.n + f : (src - 1) * p.B + b;
+    };
+
     if (threadIdx.x == 0) {
         mbar_init(bar(B_QFULL), 1);
         for (int i = 0; i < NS; ++i) {
             mbar_init(bar(B_KFULL + i), 1);
-            mbar_init(bar(B_KEMPTY + i), 1);
+            mbar_init(bar(B_KEMPTY + i), 2);
             mbar_init(bar(B_VFULL + i), 1);
             mbar_init(bar(B_VREADY + i), 1);
-            mbar_init(bar(B_VEMPTY + i), 1);
+            mbar_init(bar(B_VEMPTY + i), 2);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(B_SFULL + i), 1);
-            mbar_init(bar(B_PFULL + i), 8);
+            mbar_init(bar(B_SFREE + i), 4);
             mbar_init(bar(B_ODONE + i), 1);
-            mbar_init(bar(B_OSTAGED + i), 8);
+            mbar_init(bar(B_FIN + i), 1);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(bar(B_XCH + i), 2);
-        for (int i = 0; i < 2; ++i) mbar_init(bar(B_EXP + i), 8);
+        for (int i = 0; i < 2 * kChunks; ++i) mbar_init(bar(B_PFULL + i), 4);
+        for (int i = 0; i < kChunks; ++i) mbar_init(bar(B_PFREE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
+        // the first loads go out before TMEM allocation and the CTA-wide sync
         prefetch_tmap(&tm.q);
         prefetch_tmap(&tm.k);
         prefetch_tmap(&tm.v);
         prefetch_tmap(&tm.sk);
         prefetch_tmap(&tm.sv);
         prefetch_tmap(&tm.o);
+        mbar_expect_tx(bar(B_QFULL), 2 * tile_bytes(NKD));
+        load_tile(sb + L.q0, &tm.q, row0, b * p.n + f, bar(B_QFULL));
+        load_tile(sb + L.q0 + TB, &tm.q, row0 + kRows, b * p.n + f, bar(B_QFULL));
+        if (NB > 0) {
+            const CUtensorMap *mk, *mv;
+            int r, fr;
+            kv_src(0, mk, mv, r, fr);
+            mbar_expect_tx(bar(B_KFULL), tile_bytes(NKD));
+            load_tile(sb + L.k0, mk, r, fr, bar(B_KFULL));
+            mbar_expect_tx(bar(B_VFULL), tile_bytes(NKD));
+            load_tile(sb + L.v0, mv, r, fr, bar(B_VFULL));
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32((const void *)tmem_slot), kTmemCols);
@@ -328,69 +380,68 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     const bool ones_col = (p.D & 31) != 0;
 
     if (warp == 0) {
-        // ------------------------------- TMA producer (one thread) --------------------
-        if (lane == 0) {
-            // one operand tile: NB32 boxes of 32 columns
-            auto load_tile = [&](uint32_t dst, const CUtensorMap *map, int r0, int fr, uint32_t bar_addr) {
-                for (int a = 0; a < NB32; ++a) tma_load_4d(dst + a * 8192u, map, 32 * a, h, r0, fr, bar_addr);
-            };
-            mbar_expect_tx(bar(B_QFULL), 2 * tile_bytes(NKD));
-            load_tile(sb + L.q0, &tm.q, row0, b * p.n + f, bar(B_QFULL));
-            load_tile(sb + L.q0 + TB, &tm.q, row0 + kRows, b * p.n + f, bar(B_QFULL));
-            // V preparation (one block behind the issue): when D is not a multiple of 32,
-            // column D of the landed V tile := 1.0 (bf16 0x3F80) at its swizzled address
-            // (64-byte rows, 16-byte chunk index ^= (row >> 1) & 3); then V is ready
-            auto prep = [&](int jv) -> bool {
-                const int s = jv % NS;
-                if (!mbar_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
-                if (ones_col) {
-                    const uint32_t vt = sb + L.v0 + s * TB;
-                    const int D = p.D;
-                    const int c = (D & 31) >> 3;
-                    const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
-#pragma unroll 4
-                    for (int r = 0; r < kKeys; ++r)
-                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
-                                     "h"((unsigned short)0x3F80)
-                                     : "memory");
-                    fence_proxy_async_smem();
-                }
-                mbar_arrive(bar(B_VREADY + s));
-                return true;
-            };
-            int issued_k = -1, issued_v = -1;
-            bool ok = true;
-            for (int j = 0; ok && j < NB; ++j) {
-                const int s = j % NS;
-                const int u = j / NS;
-                const int src = j / p.nkb;
-                const int kb = j - src * p.nkb;
-                const CUtensorMap *mk = src == 0 ? &tm.k : &tm.sk;
-                const CUtensorMap *mv = src == 0 ? &tm.v : &tm.sv;
-                const int fr = src == 0 ? b * p.n + f : (src - 1) * p.B + b;
-                if (j >= NS && !mbar_wait(bar(B_KEMPTY + s), (u - 1) & 1, 201, abort_flag)) { ok = false; break; }
+        // ------------------------------- TMA producer (one warp) ----------------------
+        // lane 0 issues the loads (block 0 went out with the barrier setup); the whole
+        // warp prepares each landed V tile.
+        // V preparation (one block behind the loads): when D is not a multiple of 32,
+        // column D of the landed V tile := 1.0 (bf16 0x3F80) at its swizzled address
+        // (64-byte rows, 16-byte chunk index ^= (row >> 1) & 3), four rows per lane
+        auto prep = [&](int jv) -> bool {
+            const int s = jv % NS;
+            if (!warp_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
+            if (ones_col) {
+                const uint32_t vt = sb + L.v0 + s * TB;
+                const int D = p.D;
+                const int c = (D & 31) >> 3;
+                const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
+#pragma unroll
+                for (int r = lane; r < kKeys; r += 32)
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
+                                 "h"((unsigned short)0x3F80)
+                                 : "memory");
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_VREADY + s));
+            return true;
+        };
+        int issued_k = NB > 0 ? 0 : -1, issued_v = issued_k;
+        bool ok = true;
+        for (int j = 1; ok && j < NB; ++j) {
+            const int s = j % NS;
+            const int u = j / NS;
+            const CUtensorMap *mk, *mv;
+            int r, fr;
+            kv_src(j, mk, mv, r, fr);
+            if (j >= NS && !warp_wait(bar(B_KEMPTY + s), (u - 1) & 1, 201, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
                 mbar_expect_tx(bar(B_KFULL + s), tile_bytes(NKD));
-                load_tile(sb + L.k0 + s * TB, mk, kb * kKeys, fr, bar(B_KFULL + s));
-                issued_k = j;
-                if (j >= NS && !mbar_wait(bar(B_VEMPTY + s), (u - 1) & 1, 202, abort_flag)) { ok = false; break; }
+                load_tile(sb + L.k0 + s * TB, mk, r, fr, bar(B_KFULL + s));
+            }
+            issued_k = j;
+            if (j >= NS && !warp_wait(bar(B_VEMPTY + s), (u - 1) & 1, 202, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
                 mbar_expect_tx(bar(B_VFULL + s), tile_bytes(NKD));
-                load_tile(sb + L.v0 + s * TB, mv, kb * kKeys, fr, bar(B_VFULL + s));
-                issued_v = j;
-                if (j >= 1 && !prep(j - 1)) ok = false;
+                load_tile(sb + L.v0 + s * TB, mv, r, fr, bar(B_VFULL + s));
             }
-            if (ok && NB > 0) prep(NB - 1);
-            // wind-down after an abort: let every issued load land before the CTA exits
-            // (each ring slot's last use is the most recent phase of its barrier)
-            if (*abort_flag) {
-                mbar_wait(bar(B_QFULL), 0, 0, nullptr, 2000000ull);
-                for (int j = issued_k; j >= 0 && j > issued_k - NS; --j)
-                    mbar_wait(bar(B_KFULL + j % NS), (j / NS) & 1, 0, nullptr, 2000000ull);
-                for (int j = issued_v; j >= 0 && j > issued_v - NS; --j)
-                    mbar_wait(bar(B_VFULL + j % NS), (j / NS) & 1, 0, nullptr, 2000000ull);
-            }
+            issued_v = j;
+            if (!prep(j - 1)) ok = false;
         }
-    } else if (warp == 1) {
-        // ------------------------------- MMA issuer (one thread) -----------------------
+        if (ok && NB > 0) prep(NB - 1);
+        // wind-down after an abort: let every issued load land before the CTA exits
+        // (each ring slot's last use is the most recent phase of its barrier)
+        if (lane == 0 && *abort_flag) {
+            mbar_wait(bar(B_QFULL), 0, 0, nullptr, 2000000ull);
+            for (int j = issued_k; j >= 0 && j > issued_k - NS; --j)
+                mbar_wait(bar(B_KFULL + j % NS), (j / NS) & 1, 0, nullptr, 2000000ull);
+            for (int j = issued_v; j >= 0 && j > issued_v - NS; --j)
+                mbar_wait(bar(B_VFULL + j % NS), (j / NS) & 1, 0, nullptr, 2000000ull);
+        }
+    } else if (warp <= 2) {
+        // ------------------------- MMA issuers: warp 1 tile A, warp 2 tile B ------------
+        // One issuing thread per tile: a thread issues about one tcgen05.mma per ~100
+        // cycles whatever N is, so two issuers keep both tiles' products moving.
+        const int X = warp - 1;
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16(kRows, DP, false, true);
@@ -398,125 +449,112 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             // start-address field (addresses stay below 256 KB, so no carry leaves it).
             // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
             // MN-major (V): atoms of 32 head-dims 8 KB apart (LBO), 8-key groups 512 B apart.
-            // (stage tiles are TB bytes apart, so one base descriptor per ring suffices)
-            const uint64_t dq0 = sdesc(sb + L.q0, 16, 512, kSw64);
+            const uint64_t dq = sdesc(sb + L.q0 + X * TB, 16, 512, kSw64);
             const uint64_t dk0 = sdesc(sb + L.k0, 16, 512, kSw64);
             const uint64_t dv0 = sdesc(sb + L.v0, 8192, 512, kSw64);
             auto koff = [](int kk) -> uint64_t { return (uint64_t)(((kk >> 1) * 8192 + (kk & 1) * 32) >> 4); };
-            // S_X = Q_X K^T into TMEM columns [128 X, 128 X + 128)
-            auto issue_qk = [&](int X, int j) {
-                const uint64_t bk = dk0 + (uint64_t)(((j % NS) * TB) >> 4), bq = dq0 + (uint64_t)((X * TB) >> 4);
+            const uint32_t s_x = tmem + TM::s(X), p_x = tmem + TM::p(X), o_x = tmem + TM::o(X);
+            // S_X = Q_X K(j)^T; the commits release the scores to the softmax warps and
+            // (with the other tile's commit) the K slot to the producer
+            auto issue_qk = [&](int j) {
+                const uint64_t bk = dk0 + (uint64_t)(((j % NS) * TB) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < NKD; ++kk)
-                    tc_mma_ss(tmem + X * kKeys, bq + koff(kk), bk + koff(kk), idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(s_x, dq + koff(kk), bk + koff(kk), idesc_qk, kk > 0 ? 1u : 0u);
                 tc_commit(bar(B_SFULL + X));
+                tc_commit(bar(B_KEMPTY + j % NS));
             };
-            // O_X (+)= P_X V, P_X read from TMEM (two bf16 per column, 8 columns per 16 keys)
-            auto issue_pv = [&](int X, int j) {
+            // O_X (+)= P chunk c V(j): P holds two bf16 per column, 8 columns per 16 keys;
+            // chunk c is columns 16c..16c+15 (keys 32c..32c+31), k-steps 2c and 2c+1
+            auto issue_pv = [&](int j, int c) {
                 const uint64_t bv = dv0 + (uint64_t)(((j % NS) * TB) >> 4);
-                const uint32_t o = tmem + 2 * kKeys + X * kKeys;
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk)
-                    tc_mma_ts(o, tmem + X * kKeys + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
+                for (int e = 0; e < 2; ++e) {
+                    const int kk = 2 * c + e;
+                    tc_mma_ts(o_x, p_x + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
                               (j > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(B_ODONE + X));
+                }
             };
-            int done_a = 0, done_b = 0;   // P V products issued per tile
             bool ok = mbar_wait(bar(B_QFULL), 0, 211, abort_flag) && mbar_wait(bar(B_KFULL), 0, 212, abort_flag);
             if (ok) {
                 tc_fence_after();
-                issue_qk(0, 0);
-                issue_qk(1, 0);
-                tc_commit(bar(B_KEMPTY));
+                issue_qk(0);
             }
             for (int j = 0; ok && j < NB; ++j) {
-                const int s = j % NS;
-                const int s1 = (j + 1) % NS;
-                if (!mbar_wait(bar(B_VREADY + s), (j / NS) & 1, 213, abort_flag)) break;
-                // tile A: P_A(j) V(j), then S_A(j+1) (in issue order, so P_A is read before
-                // S_A(j+1) overwrites it)
-                if (!mbar_wait(bar(B_PFULL + 0), j & 1, 214, abort_flag)) break;
-                tc_fence_after();
-                issue_pv(0, j);
-                done_a = j + 1;
-                if (j + 1 < NB) {
-                    if (!mbar_wait(bar(B_KFULL + s1), ((j + 1) / NS) & 1, 215, abort_flag)) break;
+                if (kSharedP && j + 1 < NB) {
+                    // the tile's score region is free once its softmax warps have read
+                    // S(j): compute S(j+1) while they exponentiate
+                    const int j1 = j + 1;
+                    if (!mbar_wait(bar(B_SFREE + X), j & 1, 213, abort_flag) ||
+                        !mbar_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag))
+                        break;
                     tc_fence_after();
-                    issue_qk(0, j + 1);
+                    issue_qk(j1);
                 }
-                // tile B
-                if (!mbar_wait(bar(B_PFULL + 1), j & 1, 216, abort_flag)) break;
-                tc_fence_after();
-                issue_pv(1, j);
-                tc_commit(bar(B_VEMPTY + s));
-                done_b = j + 1;
-                if (j + 1 < NB) {
-                    issue_qk(1, j + 1);
-                    tc_commit(bar(B_KEMPTY + s1));
+                if (!mbar_wait(bar(B_VREADY + j % NS), (j / NS) & 1, 215, abort_flag)) break;
+                bool okc = true;
+                for (int c = 0; c < kChunks; ++c) {
+                    if (!mbar_wait(bar(B_PFULL + kChunks * X + c), j & 1, 216, abort_flag)) { okc = false; break; }
+                    tc_fence_after();
+                    issue_pv(j, c);
+                    if (kSharedP) tc_commit(bar(B_PFREE + c));
+                }
+                if (!okc) break;
+                tc_commit(bar(B_ODONE + X));
+                tc_commit(bar(B_VEMPTY + j % NS));
+                if (!kSharedP && j + 1 < NB) {
+                    // P was written over S: the next scores follow the P V product
+                    const int j1 = j + 1;
+                    if (!mbar_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag)) break;
+                    tc_fence_after();
+                    issue_qk(j1);
                 }
             }
             // wind-down: the tensor core must be idle before TMEM is released
-            if (done_a > 0) mbar_wait(bar(B_ODONE + 0), (done_a - 1) & 1, 0, nullptr, 2000000ull);
-            if (done_b > 0) mbar_wait(bar(B_ODONE + 1), (done_b - 1) & 1, 0, nullptr, 2000000ull);
+            tc_commit(bar(B_FIN + X));
+            mbar_wait(bar(B_FIN + X), 0, 0, nullptr, 2000000ull);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= kSoftmaxWarp0) {
         // ------------------------------- softmax / epilogue ---------------------------
-        // 16 warps (2..17): tile X = sw / 8, half hh = (sw / 4) % 2 of a block's 128 keys,
-        // lane quarter = warp % 4 (each group of four consecutive warps covers all four).
-        // The two threads of a query row (same lane, warps sw and sw ^ 4) exchange their
-        // partial row maxima through shared memory once per block.
-        const int sw = warp - 2;
-        const int X = sw >> 3;
-        const int hh = (sw >> 2) & 1;
+        // 8 warps: tile X = (warp - 4) / 4, lane quarter = warp % 4, one thread per query
+        // row (its TMEM lane), all 128 keys of a block in its registers.
+        const int sw = warp - kSoftmaxWarp0;
+        const int X = sw >> 2;
         const int quarter = warp & 3;                     // TMEM lanes 32*quarter ..
         const int row = quarter * 32 + lane;              // query row of this thread in its tile
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
-        const uint32_t s_col = tmem + lane_bits + X * kKeys;
-        const uint32_t o_col = tmem + lane_bits + 2 * kKeys + X * kKeys;
-        const uint32_t xch = bar(B_XCH + X * 4 + quarter);
-        float *red = reinterpret_cast<float *>(sgen + L.red);   // [parity][tile][half][row]
-        auto red_at = [&](int par, int half) -> float & { return red[((par * 2 + X) * 2 + half) * kRows + row]; };
+        const uint32_t s_col = tmem + lane_bits + TM::s(X);
+        const uint32_t p_col = tmem + lane_bits + TM::p(X);
+        const uint32_t o_col = tmem + lane_bits + TM::o(X);
         const float neg_inf = __int_as_float(0xff800000);
         const float scale = p.scale_log2;
         float m_used = neg_inf;     // max (log2 units) the probabilities are taken against
-        float l_sum = 0.f;         // partial row sum, kept only when there is no padding column
+        float l_sum = 0.f;         // row sum, kept only when there is no padding column
         bool ok = true;
-        int nx = 0;                 // exchanges done (phase counter of xch)
-        // exchange one float with the row's partner thread; false if the wait gave up
-        auto exchange = [&](float mine, float &theirs) -> bool {
-            red_at(nx & 1, hh) = mine;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xch);
-            if (!warp_wait(xch, nx & 1, 226, abort_flag)) return false;
-            theirs = red_at(nx & 1, hh ^ 1);
-            ++nx;
-            return true;
-        };
-        for (int j = 0; j < NB; ++j) {
+        for (int j = 0; ok && j < NB; ++j) {
             const int kb = j % p.nkb;
-            const int valid = min(kKeys, p.HW - kb * kKeys) - 64 * hh;   // valid keys of this half
-            // S_X(j) ready; its commit also covers the previous P V of this tile
+            const int valid = min(kKeys, p.HW - kb * kKeys);   // valid keys of this block
             if (!warp_wait(bar(B_SFULL + X), j & 1, 221, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            // pass 1: this half's 64 scores into registers, partial row max, exchange
-            uint32_t sr[64];
-            tmem_ld64(s_col + 64 * hh, sr);
+            // the block's 128 scores into registers; then the score region is free
+            uint32_t sr[128];
+            tmem_ld128(s_col, sr);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SFREE + X));
             float m8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = neg_inf;
-            if (valid >= 64) {
+            if (valid >= kKeys) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
+                for (int i = 0; i < kKeys; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
             } else {
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
+                for (int i = 0; i < kKeys; ++i)
                     if (i < valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
             }
-            const float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            float qm;
-            if (!exchange(pm, qm)) { ok = false; break; }
-            const float mx = fmaxf(pm, qm) * scale;
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale;
             float alpha = 1.f;
             const bool upd = mx > m_used + kLazyRescale;
             if (upd) {
@@ -524,11 +562,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 m_used = mx;
             }
             if (j > 0 && __any_sync(0xffffffffu, upd)) {
-                // this thread's half of the row's O columns
+                // the previous block's P V must be done accumulating before O is rescaled
+                if (!warp_wait(bar(B_ODONE + X), (j - 1) & 1, 228, abort_flag)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < DP / 32; ++c) {
+                for (int c = 0; c < DP / 16; ++c) {
                     uint32_t o[16];
-                    const uint32_t a = o_col + (uint32_t)(hh * (DP / 2) + 16 * c);
+                    const uint32_t a = o_col + (uint32_t)(16 * c);
                     tmem_ld16(a, o);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
@@ -536,44 +576,50 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 }
             }
             l_sum *= alpha;
-            // The two tiles take turns on the exponential unit (16 lanes/clock/SM, the
-            // scarce pipe): tile B's block j waits for tile A's block j, tile A's block
-            // j+1 for tile B's block j, so each tile's products run on the tensor core
-            // while the other tile exponentiates.
-            if (X == 1 || j > 0) {
-                const int other_j = X == 1 ? j : j - 1;
-                if (!warp_wait(bar(B_EXP + (X ^ 1)), other_j & 1, 227, abort_flag)) { ok = false; break; }
-            }
-            // pass 2: probabilities from the registers, written over the scores in TMEM as
-            // bf16 pairs (keys 64 hh + 32 c .. go to columns 32 hh + 16 c ..)
+            // probabilities from the registers as bf16 pairs (keys 32c.. -> P columns
+            // 16c..), handed to the issuer one chunk at a time; a chunk's store completes
+            // while the next chunk's exponentials run
             const float neg_m = -m_used;
-            float ls = 0.f;
+            const int use = 2 * j + X;    // turn of this tile on the shared P region
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < kChunks; ++c) {
                 uint32_t w[16];
+                float ls = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int k0 = 32 * c + 2 * i;
                     float e0 = ex2(fmaf(__uint_as_float(sr[k0]), scale, neg_m));
                     float e1 = ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale, neg_m));
-                    if (valid < 64) {
+                    if (valid < kKeys) {
                         if (k0 >= valid) e0 = 0.f;
                         if (k0 + 1 >= valid) e1 = 0.f;
                     }
                     w[i] = pack_bf16x2(e0, e1);
                     if (!ones_col) ls += bf16_lo(w[i]) + bf16_hi(w[i]);
                 }
-                tmem_st16(s_col + (uint32_t)(32 * hh + 16 * c), w);
+                l_sum += ls;
+                if (c > 0) {
+                    // the previous chunk has landed: hand it over
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + c - 1));
+                }
+                if (kSharedP && use > 0) {
+                    // the other tile's P V products must be done reading this chunk
+                    if (!warp_wait(bar(B_PFREE + c), (use - 1) & 1, 229, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                tmem_st16(p_col + (uint32_t)(16 * c), w);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_EXP + X));
-            l_sum += ls;
+            if (!ok) break;
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_PFULL + X));
+            if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + kChunks - 1));
         }
-        // ---- epilogue: O / l -> bf16 -> shared (dense [128][D]) -> one TMA store -------
+        // ---- epilogue: O / l -> bf16 rows staged in the tile's (now unused) Q buffer,
+        //      then one TMA store of the warp's 32 rows -----------------------------------
         if (ok && warp_wait(bar(B_ODONE + X), (NB - 1) & 1, 224, abort_flag)) {
             tc_fence_after();
             float l = l_sum;
@@ -583,41 +629,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     if (i == (p.D & 15)) l = __uint_as_float(o[i]);
-            } else {
-                float lt = 0.f;
-                if (!exchange(l_sum, lt)) ok = false;
-                l = l_sum + lt;
             }
             const float inv = 1.f / l;
             uint8_t *orow = sgen + L.q0 + X * TB + (size_t)row * (size_t)(p.D * 2);
 #pragma unroll
-            for (int c = 0; c < DP / 32; ++c) {
-                const int col = hh * (DP / 2) + 16 * c;   // first head-dim of this chunk
+            for (int c = 0; c < DP / 16; ++c) {
                 uint32_t o[16];
-                tmem_ld16(o_col + (uint32_t)col, o);
+                tmem_ld16(o_col + (uint32_t)(16 * c), o);
 #pragma unroll
                 for (int hlf = 0; hlf < 2; ++hlf) {
-                    if (col + 8 * hlf < p.D) {
+                    const int col = 16 * c + 8 * hlf;
+                    if (col < p.D) {
                         auto v = [&](int i) { return __uint_as_float(o[8 * hlf + i]) * inv; };
                         uint4 w;
                         w.x = pack_bf16x2(v(0), v(1));
                         w.y = pack_bf16x2(v(2), v(3));
                         w.z = pack_bf16x2(v(4), v(5));
                         w.w = pack_bf16x2(v(6), v(7));
-                        *reinterpret_cast<uint4 *>(orow + 2 * col + 16 * hlf) = w;
+                        *reinterpret_cast<uint4 *>(orow + 2 * col) = w;
                     }
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(B_OSTAGED + X));
-        }
-        // tile rows entirely past HW are not stored
-        if (sw == 8 * X && lane == 0 && row0 + X * kRows < p.HW &&
-            mbar_wait(bar(B_OSTAGED + X), 0, 225, abort_flag)) {
-            tma_store_4d(&tm.o, sb + L.q0 + X * TB, 0, h, row0 + X * kRows, b * p.n + f);
-            bulk_commit();
-            bulk_wait_read<0>();
+            // rows past HW are not written by the TMA unit; a box starting past HW is skipped
+            const int r0 = row0 + X * kRows + quarter * 32;
+            if (lane == 0 && r0 < p.HW) {
+                tma_store_4d(&tm.o, sb + L.q0 + X * TB + (uint32_t)(quarter * 32 * p.D * 2), 0, h, r0,
+                             b * p.n + f);
+                bulk_commit();
+                bulk_wait_read<0>();
+            }
         }
     }
     tc_fence_before();

@@ -176,6 +176,27 @@ def test_ragged_shapes(shape):
         lp.ar_step(wl.chunk_len - 1, 1)
 
 
+@pytest.mark.parametrize("head_dim", [72, 64, 128])
+def test_spatial_max_grows_in_late_blocks(head_dim):
+    """Spatial-cache keys scaled up (more for later cache frames and for the second key
+    block of each frame), so the running row max jumps well past the lazy-rescale
+    threshold after the first blocks and O is rescaled between P V products."""
+    from ca2_synth import bf16_bits, bf16_to_f32
+    from tests.gpu_util import Loop
+    wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, hw=256, heads=2, head_dim=head_dim,
+             batch=1, chunk_len=3, p_max=6, p_spatial=3)
+    lp = Loop(wl, seed=21)
+    kt, vt = lp.gen.frames(3), lp.gen.frames(3)
+    ks = bf16_to_f32(lp.gen.frames(3)).copy()
+    for i in range(3):
+        ks[:, i] *= 3.0 * (i + 1)
+    ks[:, :, 128:] *= 2.0
+    vs = lp.gen.frames(3)
+    lp.write([kt], [vt], [bf16_bits(ks)], [vs])
+    q, k, v = lp.gen.qkv(3)
+    lp.spatial(0, q, k, v, use_prefix=1)
+
+
 def test_multi_layer_write_bit_exact():
     """One cache-write launch for many layers (more than one launch's layer table)."""
     from tests.gpu_util import Loop
