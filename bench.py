@@ -198,24 +198,32 @@ def run_ca2(args):
 
     def capture(use_prefix, timed):
         """One pass over the 28 blocks (spatial then temporal attention per block) captured
-        into a CUDA graph.  A timed capture brackets every kernel with event-record nodes,
-        so per-kernel device times come from the replay itself, with no host gaps."""
+        into a CUDA graph.  A timed capture groups the pass by kernel instead: the 28
+        spatial launches between two event nodes, then the 28 temporal launches before a
+        third, so each kernel's mean device time is measured without host gaps or per-launch
+        event overhead (the synthetic inputs of different calls do not depend on each other,
+        so the order within a pass does not change the work)."""
         graph = torch.cuda.CUDAGraph()
         evs = []
         with torch.cuda.stream(cap):
             graph.capture_begin()
-            for L in range(NL):
-                p = P[L]
-                if timed:
-                    e0, e1, e2 = (torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
-                    e0.record(cap)
-                spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, cap_sp)
-                if timed:
-                    e1.record(cap)
-                tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, cap_sp)
-                if timed:
-                    e2.record(cap)
-                    evs.append(("den" if use_prefix else "self", e0, e1, e2))
+            if timed:
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
+                e0.record(cap)
+                for L in range(NL):
+                    p = P[L]
+                    spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, cap_sp)
+                e1.record(cap)
+                for L in range(NL):
+                    p = P[L]
+                    tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, cap_sp)
+                e2.record(cap)
+                evs.append(("den" if use_prefix else "self", e0, e1, e2))
+            else:
+                for L in range(NL):
+                    p = P[L]
+                    spat(h, L, p["sq"], p["sk"], p["sv"], SO[L], l, use_prefix, cap_sp)
+                    tempo(h, L, p["tq"], p["tk"], p["tv"], TO[L], l, cap_sp)
             graph.capture_end()
         live_graphs.append(graph)
         return graph, evs
@@ -224,8 +232,9 @@ def run_ca2(args):
         """One AR step: TPE indices, T denoising passes, the cache-writing pass, evict, write.
 
         The queue state is fixed until the write, so each pass is a CUDA graph captured
-        once per step.  Pass 0 and the cache-writing pass replay timed graphs (event nodes
-        around every kernel); passes 1..T-1 replay the plain denoising graph."""
+        once per step.  Pass 0 and the cache-writing pass replay timed graphs (launches
+        grouped by kernel between event nodes); passes 1..T-1 replay the plain denoising
+        graph."""
         ca2.ca2_tpe_indices(h, g0[0], 0, l)
         g_den, _ = capture(1, False)
         g_den_t, e_den = capture(1, True)
@@ -284,8 +293,8 @@ def run_ca2(args):
         if kind == "write":
             wr_ms.append(a.elapsed_time(b_))
             continue
-        (sp_den if kind == "den" else sp_self).append(a.elapsed_time(b_))
-        tp_ms.append(b_.elapsed_time(c))
+        (sp_den if kind == "den" else sp_self).append(a.elapsed_time(b_) / NL)
+        tp_ms.append(b_.elapsed_time(c) / NL)
     resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * plane) * 2 / 1e9
     launches_per_step = (T + 1) * NL * 2 + 1
     tokens_per_step = (T + 1) * NL * B * l * HW

@@ -12,22 +12,23 @@
 //                independent rings (K is released as soon as both QK^T products have read
 //                it, V after both P V products).  An operand tile is ceil(D/32) boxes of 32
 //                head-dims x 128 tokens (64-byte rows, 64-byte swizzle); columns past D
-//                (72 -> 96) and rows past HW are zero-filled by the TMA unit.  One block
-//                behind its loads the warp prepares each landed V tile: when D is not a
-//                multiple of 32, padding column D is set to 1.0, so the P V product also
-//                accumulates the row sum of the probabilities into O[:, D].
+//                (72 -> 96) and rows past HW are zero-filled by the TMA unit.  When D is
+//                not a multiple of 32, padding column D of each landed V tile is set to 1.0
+//                (by warp 3), so the P V product also accumulates the row sum of the
+//                probabilities into O[:, D].
 //   warps 1, 2   MMA issuers of tile A and tile B (one thread each; warp 1 owns the 512
 //                TMEM columns).  A single thread issues about one tcgen05.mma per ~100
 //                cycles whatever the tile width, so each tile has its own issuer.  The
 //                tile's next QK^T is issued as soon as its softmax warps have read the
 //                current scores, and its P V product chunk by chunk as the probabilities
 //                land, so the tensor core works while the exponentials run.
-//   warp 3       idle.
+//   warp 3       prepares each landed V tile (the padding column of ones, below).
 //   warps 4-11   softmax: 4 warps per tile, one thread per query row (its TMEM lane; warp
 //                % 4 selects the lane quarter) holding all 128 scores of a block in
 //                registers, so the row max needs no exchange.  The exponential unit
-//                (measured 16 lanes/clock/SM) is the scarce pipe.  The two tiles fill one
-//                shared TMEM probability region in turns, chunk by chunk, each turn
+//                (measured 16 lanes/clock/SM) is the scarce pipe; both tiles' warps share
+//                it, so one warp's stalls are filled by the other's work.  The tiles fill
+//                one shared TMEM probability region in turns, chunk by chunk, each turn
 //                waiting for the P V products of the previous one.  The running max moves
 //                only when it grows by more than 2^8 (O is then rescaled in TMEM).  The
 //                bf16 probabilities are the A operand of the P V product, read from TMEM.
@@ -95,6 +96,41 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Warp-wide forms: every lane of the warp executes the statement with warp-uniform
+// operands and one elected lane issues.  Operands the compiler can prove uniform keep the
+// issue cost near the tensor core's own rate (a single divergent lane with operands in
+// per-thread registers measured about 100 cycles per instruction).
+__device__ __forceinline__ void tc_mma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, -1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, -1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_w(uint32_t bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, -1;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
         : "memory");
 }
 
@@ -318,10 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     auto load_tile = [&](uint32_t dst, const CUtensorMap *map, int r0, int fr, uint32_t bar_addr) {
         for (int a = 0; a < NB32; ++a) tma_load_4d(dst + a * 8192u, map, 32 * a, h, r0, fr, bar_addr);
     };
-    // key block j -> (tensor map, first key row, frame index)
+    // key block j -> (tensor map, first key row, frame index).  The spatial-cache frames
+    // come first and the own frame last: cache frames are shared by the n frames' CTAs
+    // (mostly L2 hits), so the first blocks arrive quickly, and the own frame's blocks,
+    // unique to this CTA and read from HBM, stream in while the cache blocks are computed.
+    // The order only changes the summation order of the online softmax.
     auto kv_src = [&](int j, const CUtensorMap *&mk, const CUtensorMap *&mv, int &r, int &fr) {
-        const int src = j / p.nkb;
-        r = (j - src * p.nkb) * kKeys;
+        const int si = j / p.nkb;
+        const int src = p.n_src > 1 ? (si + 1) % p.n_src : 0;
+        r = (j - si * p.nkb) * kKeys;
         mk = src == 0 ? &tm.k : &tm.sk;
         mv = src == 0 ? &tm.v : &tm.sv;
         fr = src == 0 ? b * p.n + f : (src - 1) * p.B + b;
@@ -381,30 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
 
     if (warp == 0) {
         // ------------------------------- TMA producer (one warp) ----------------------
-        // lane 0 issues the loads (block 0 went out with the barrier setup); the whole
-        // warp prepares each landed V tile.
-        // V preparation (one block behind the loads): when D is not a multiple of 32,
-        // column D of the landed V tile := 1.0 (bf16 0x3F80) at its swizzled address
-        // (64-byte rows, 16-byte chunk index ^= (row >> 1) & 3), four rows per lane
-        auto prep = [&](int jv) -> bool {
-            const int s = jv % NS;
-            if (!warp_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
-            if (ones_col) {
-                const uint32_t vt = sb + L.v0 + s * TB;
-                const int D = p.D;
-                const int c = (D & 31) >> 3;
-                const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
-#pragma unroll
-                for (int r = lane; r < kKeys; r += 32)
-                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
-                                 "h"((unsigned short)0x3F80)
-                                 : "memory");
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_VREADY + s));
-            return true;
-        };
+        // lane 0 issues the loads (block 0 went out with the barrier setup) as fast as
+        // ring slots free up.
         int issued_k = NB > 0 ? 0 : -1, issued_v = issued_k;
         bool ok = true;
         for (int j = 1; ok && j < NB; ++j) {
@@ -425,9 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 load_tile(sb + L.v0 + s * TB, mv, r, fr, bar(B_VFULL + s));
             }
             issued_v = j;
-            if (!prep(j - 1)) ok = false;
         }
-        if (ok && NB > 0) prep(NB - 1);
         // wind-down after an abort: let every issued load land before the CTA exits
         // (each ring slot's last use is the most recent phase of its barrier)
         if (lane == 0 && *abort_flag) {
@@ -439,81 +456,106 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         }
     } else if (warp <= 2) {
         // ------------------------- MMA issuers: warp 1 tile A, warp 2 tile B ------------
-        // One issuing thread per tile: a thread issues about one tcgen05.mma per ~100
-        // cycles whatever N is, so two issuers keep both tiles' products moving.
+        // The whole warp runs the loop with warp-uniform operands; one elected lane issues.
         const int X = warp - 1;
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16(kRows, DP, false, true);
-            // Descriptors are built once; a k-step only adds its byte offset / 16 to the
-            // start-address field (addresses stay below 256 KB, so no carry leaves it).
-            // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
-            // MN-major (V): atoms of 32 head-dims 8 KB apart (LBO), 8-key groups 512 B apart.
-            const uint64_t dq = sdesc(sb + L.q0 + X * TB, 16, 512, kSw64);
-            const uint64_t dk0 = sdesc(sb + L.k0, 16, 512, kSw64);
-            const uint64_t dv0 = sdesc(sb + L.v0, 8192, 512, kSw64);
-            auto koff = [](int kk) -> uint64_t { return (uint64_t)(((kk >> 1) * 8192 + (kk & 1) * 32) >> 4); };
-            const uint32_t s_x = tmem + TM::s(X), p_x = tmem + TM::p(X), o_x = tmem + TM::o(X);
-            // S_X = Q_X K(j)^T; the commits release the scores to the softmax warps and
-            // (with the other tile's commit) the K slot to the producer
-            auto issue_qk = [&](int j) {
-                const uint64_t bk = dk0 + (uint64_t)(((j % NS) * TB) >> 4);
+        const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+        constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16(kRows, DP, false, true);
+        // Descriptors are built once; a k-step only adds its byte offset / 16 to the
+        // start-address field (addresses stay below 256 KB, so no carry leaves it).
+        // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
+        // MN-major (V): atoms of 32 head-dims 8 KB apart (LBO), 8-key groups 512 B apart.
+        const uint64_t dq = sdesc(sb + L.q0 + X * TB, 16, 512, kSw64);
+        const uint64_t dk0 = sdesc(sb + L.k0, 16, 512, kSw64);
+        const uint64_t dv0 = sdesc(sb + L.v0, 8192, 512, kSw64);
+        auto koff = [](int kk) -> uint64_t { return (uint64_t)(((kk >> 1) * 8192 + (kk & 1) * 32) >> 4); };
+        const uint32_t s_x = tm_u + TM::s(X), p_x = tm_u + TM::p(X), o_x = tm_u + TM::o(X);
+        // S_X = Q_X K(j)^T; the commits release the scores to the softmax warps and
+        // (with the other tile's commit) the K slot to the producer
+        auto issue_qk = [&](int j) {
+            const uint64_t bk = dk0 + (uint64_t)(((j % NS) * TB) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < NKD; ++kk)
-                    tc_mma_ss(s_x, dq + koff(kk), bk + koff(kk), idesc_qk, kk > 0 ? 1u : 0u);
-                tc_commit(bar(B_SFULL + X));
-                tc_commit(bar(B_KEMPTY + j % NS));
-            };
-            // O_X (+)= P chunk c V(j): P holds two bf16 per column, 8 columns per 16 keys;
-            // chunk c is columns 16c..16c+15 (keys 32c..32c+31), k-steps 2c and 2c+1
-            auto issue_pv = [&](int j, int c) {
-                const uint64_t bv = dv0 + (uint64_t)(((j % NS) * TB) >> 4);
+            for (int kk = 0; kk < NKD; ++kk)
+                tc_mma_ss_w(s_x, dq + koff(kk), bk + koff(kk), idesc_qk, kk > 0 ? 1u : 0u);
+            tc_commit_w(bar(B_SFULL + X));
+            tc_commit_w(bar(B_KEMPTY + j % NS));
+        };
+        // O_X (+)= P chunk c V(j): P holds two bf16 per column, 8 columns per 16 keys;
+        // chunk c is columns 16c..16c+15 (keys 32c..32c+31), k-steps 2c and 2c+1
+        auto issue_pv = [&](int j, int c) {
+            const uint64_t bv = dv0 + (uint64_t)(((j % NS) * TB) >> 4);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int kk = 2 * c + e;
-                    tc_mma_ts(o_x, p_x + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
-                              (j > 0 || kk > 0) ? 1u : 0u);
-                }
-            };
-            bool ok = mbar_wait(bar(B_QFULL), 0, 211, abort_flag) && mbar_wait(bar(B_KFULL), 0, 212, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_qk(0);
+            for (int e = 0; e < 2; ++e) {
+                const int kk = 2 * c + e;
+                tc_mma_ts_w(o_x, p_x + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
+                            (j > 0 || kk > 0) ? 1u : 0u);
             }
-            for (int j = 0; ok && j < NB; ++j) {
-                if (kSharedP && j + 1 < NB) {
-                    // the tile's score region is free once its softmax warps have read
-                    // S(j): compute S(j+1) while they exponentiate
-                    const int j1 = j + 1;
-                    if (!mbar_wait(bar(B_SFREE + X), j & 1, 213, abort_flag) ||
-                        !mbar_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag))
-                        break;
-                    tc_fence_after();
-                    issue_qk(j1);
-                }
-                if (!mbar_wait(bar(B_VREADY + j % NS), (j / NS) & 1, 215, abort_flag)) break;
-                bool okc = true;
-                for (int c = 0; c < kChunks; ++c) {
-                    if (!mbar_wait(bar(B_PFULL + kChunks * X + c), j & 1, 216, abort_flag)) { okc = false; break; }
-                    tc_fence_after();
-                    issue_pv(j, c);
-                    if (kSharedP) tc_commit(bar(B_PFREE + c));
-                }
-                if (!okc) break;
-                tc_commit(bar(B_ODONE + X));
-                tc_commit(bar(B_VEMPTY + j % NS));
-                if (!kSharedP && j + 1 < NB) {
-                    // P was written over S: the next scores follow the P V product
-                    const int j1 = j + 1;
-                    if (!mbar_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag)) break;
-                    tc_fence_after();
-                    issue_qk(j1);
-                }
-            }
-            // wind-down: the tensor core must be idle before TMEM is released
-            tc_commit(bar(B_FIN + X));
-            mbar_wait(bar(B_FIN + X), 0, 0, nullptr, 2000000ull);
+        };
+        bool ok = warp_wait(bar(B_QFULL), 0, 211, abort_flag) && warp_wait(bar(B_KFULL), 0, 212, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            issue_qk(0);
         }
+        for (int j = 0; ok && j < NB; ++j) {
+            if (kSharedP && j + 1 < NB) {
+                // the tile's score region is free once its softmax warps have read S(j):
+                // compute S(j+1) while they exponentiate
+                const int j1 = j + 1;
+                if (!warp_wait(bar(B_SFREE + X), j & 1, 213, abort_flag) ||
+                    !warp_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag))
+                    break;
+                tc_fence_after();
+                issue_qk(j1);
+            }
+            if (!warp_wait(bar(B_VREADY + j % NS), (j / NS) & 1, 215, abort_flag)) break;
+            bool okc = true;
+            for (int c = 0; c < kChunks; ++c) {
+                if (!warp_wait(bar(B_PFULL + kChunks * X + c), j & 1, 216, abort_flag)) { okc = false; break; }
+                tc_fence_after();
+                issue_pv(j, c);
+                if (kSharedP) tc_commit_w(bar(B_PFREE + c));
+            }
+            if (!okc) break;
+            tc_commit_w(bar(B_ODONE + X));
+            tc_commit_w(bar(B_VEMPTY + j % NS));
+            if (!kSharedP && j + 1 < NB) {
+                // P was written over S: the next scores follow the P V product
+                const int j1 = j + 1;
+                if (!warp_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag)) break;
+                tc_fence_after();
+                issue_qk(j1);
+            }
+        }
+        // wind-down: the tensor core must be idle before TMEM is released
+        tc_commit_w(bar(B_FIN + X));
+        mbar_wait(bar(B_FIN + X), 0, 0, nullptr, 2000000ull);
+        __syncwarp();
+    } else if (warp == 3) {
+        // ------------------------------- V preparation (one warp) ---------------------
+        // When D is not a multiple of 32, column D of each landed V tile := 1.0 (bf16
+        // 0x3F80) at its swizzled address (64-byte rows, 16-byte chunk index ^= (row >> 1)
+        // & 3), four rows per lane; then the tile is ready for the P V products
+        auto prep = [&](int jv) -> bool {
+            const int s = jv % NS;
+            if (!warp_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
+            if (ones_col) {
+                const uint32_t vt = sb + L.v0 + s * TB;
+                const int D = p.D;
+                const int c = (D & 31) >> 3;
+                const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
+#pragma unroll
+                for (int r = lane; r < kKeys; r += 32)
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
+                                 "h"((unsigned short)0x3F80)
+                                 : "memory");
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_VREADY + s));
+            return true;
+        };
+        for (int j = 0; j < NB; ++j)
+            if (!prep(j)) break;
     } else if (warp >= kSoftmaxWarp0) {
         // ------------------------------- softmax / epilogue ---------------------------
         // 8 warps: tile X = (warp - 4) / 4, lane quarter = warp % 4, one thread per query
@@ -583,18 +625,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             const int use = 2 * j + X;    // turn of this tile on the shared P region
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
+                // all 32 exponentials of the chunk first, so that a warp keeps many in
+                // flight on the exponential unit, then the bf16 packing
+                float e[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) e[i] = ex2(fmaf(__uint_as_float(sr[32 * c + i]), scale, neg_m));
+                if (valid < kKeys) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i >= valid) e[i] = 0.f;
+                }
                 uint32_t w[16];
                 float ls = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int k0 = 32 * c + 2 * i;
-                    float e0 = ex2(fmaf(__uint_as_float(sr[k0]), scale, neg_m));
-                    float e1 = ex2(fmaf(__uint_as_float(sr[k0 + 1]), scale, neg_m));
-                    if (valid < kKeys) {
-                        if (k0 >= valid) e0 = 0.f;
-                        if (k0 + 1 >= valid) e1 = 0.f;
-                    }
-                    w[i] = pack_bf16x2(e0, e1);
+                    w[i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
                     if (!ones_col) ls += bf16_lo(w[i]) + bf16_hi(w[i]);
                 }
                 l_sum += ls;
