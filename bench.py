@@ -135,6 +135,22 @@ def committed_traffic(kernel_file: str):
     return None
 
 
+def max_over_ranks(ms: float, dist, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own device-timed milliseconds and
+    all receive the maximum (a no-op on one rank)."""
+    if world <= 1:
+        return ms
+    import torch
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(tokens_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Query tokens per second of the whole job: every rank's tokens over the slowest rank's time."""
+    return tokens_per_step * steps * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------------------------
 def run_ca2(args):
     import torch
@@ -279,11 +295,7 @@ def run_ca2(args):
         dist.barrier()
     clk = clocks.stop()
     live_graphs.clear()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, world, dev)
     st = ca2.ca2_device_status()
     if st != 0:
         raise RuntimeError("device status %d after the timed region" % st)
@@ -298,7 +310,7 @@ def run_ca2(args):
     resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * plane) * 2 / 1e9
     launches_per_step = (T + 1) * NL * 2 + 1
     tokens_per_step = (T + 1) * NL * B * l * HW
-    value = tokens_per_step * args.steps * world / (ms / 1e3)
+    value = whole_job_rate(tokens_per_step, args.steps, world, ms)
 
     # ---- roofline of each kernel ----
     pk, pk_kind = peaks()
@@ -397,12 +409,8 @@ def run_e2e(args, cache, inp, so, to, step_fn, stream, NL, tokens_per_step, worl
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    return {"value": tokens_per_step * steps * world / (ms / 1e3), "unit": "query-tokens/s",
+    ms = max_over_ranks(a.elapsed_time(b), dist, world, "cuda")
+    return {"value": whole_job_rate(tokens_per_step, steps, world, ms), "unit": "query-tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps}
 
