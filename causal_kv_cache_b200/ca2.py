@@ -228,7 +228,7 @@ def ca2_last_error_string() -> str:
 class KVCache:
     """Cache buffers allocated with torch on the current CUDA device, plus the handle.
 
-    ``ring(layer, kv)`` ([B][HW][Pmax][H][D]) and ``spatial(layer, kv)`` ([P'][B][HW][H][D])
+    ``ring(layer, kv)`` ([B][HW][H][Pmax][D]) and ``spatial(layer, kv)`` ([P'][B][HW][H][D])
     are bf16 views of the buffers with the layout documented in include/ca2.h.
     """
 
@@ -254,11 +254,11 @@ class KVCache:
             pass
 
     def ring(self, layer: int, kv: int):
-        """Token-major ring of one layer: [B][HW][Pmax][H][D]."""
+        """Ring of one layer, token-major and head-major within a token: [B][HW][H][Pmax][D]."""
         c = self.cfg
         per = c.p_max * c.batch * c.hw * c.heads * c.head_dim
         off = (layer * 2 + kv) * per
-        return self.tbuf[off:off + per].view(c.batch, c.hw, c.p_max, c.heads, c.head_dim)
+        return self.tbuf[off:off + per].view(c.batch, c.hw, c.heads, c.p_max, c.head_dim)
 
     def spatial(self, layer: int, kv: int):
         c = self.cfg

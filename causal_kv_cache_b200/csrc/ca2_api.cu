@@ -222,6 +222,8 @@ int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t
     p.sbuf = reinterpret_cast<uint4 *>(c->sbuf);
     p.row_vec = (long long)g.heads * g.head_dim / 8;   // 16-byte vectors per (video, token, frame) row
     p.tokens = (long long)g.batch * g.hw;
+    p.head_vec = g.head_dim / 8;                       // 16-byte vectors per head row
+    p.heads = g.heads;
     p.hw = g.hw;
     p.n = n;
     p.slot0 = (c->head + c->count) % g.p_max;
@@ -271,25 +273,23 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
     for (int i = 0; i < c->count; ++i) p.ring_box_mask |= 1u << (((c->head + i) % g.p_max) / 16);
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
 
-    // temporal tensors are token-major: chunk [B][HW][n][C], ring [B][HW][Pmax][C], C = H*D
+    // temporal chunk tensors are token-major [B][HW][n][H][D] (C = H*D), read as TMA boxes;
+    // the ring [B][HW][H][Pmax][D] is read with bulk copies of one head's consecutive slots
     const long long C = (long long)g.heads * g.head_dim;
+    p.rk = layer_ring(c, layer, 0);
+    p.rv = layer_ring(c, layer, 1);
     ca2::TemporalMaps m;
     const bool ok =
         encode_5d(&m.q, q, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 8, G) &&
         encode_5d(&m.k, k, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 16, G) &&
-        encode_5d(&m.v, v, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 16, G) &&
-        encode_5d(&m.rk, layer_ring(c, layer, 0), g.head_dim, g.p_max, g.heads, g.hw, g.batch, C, g.p_max * C,
-                  (long long)g.hw * g.p_max * C, 16, G) &&
-        encode_5d(&m.rv, layer_ring(c, layer, 1), g.head_dim, g.p_max, g.heads, g.hw, g.batch, C, g.p_max * C,
-                  (long long)g.hw * g.p_max * C, 16, G);
+        encode_5d(&m.v, v, g.head_dim, n, g.heads, g.hw, g.batch, C, n * C, (long long)g.hw * n * C, 16, G);
     if (!ok) {
         g_last_cuda_error = "tensor-map encoding failed";
         return CA2_ERR_CUDA;
     }
-    const int sms = sm_count();
-    if (sms <= 0) return CA2_ERR_CUDA;
-    int grid = 2 * sms;
-    if (grid > p.n_items) grid = p.n_items;
+    // one CTA per work item; the resident CTAs take over the items of CTAs that have not
+    // started (cluster launch control), so the grid's size only fixes the work list
+    const int grid = p.n_items;
     return cuda_status(ca2::launch_temporal(m, p, grid, static_cast<cudaStream_t>(stream)));
 }
 

@@ -99,6 +99,32 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int sit
     return __all_sync(0xffffffffu, ok);
 }
 
+// ---- work stealing between CTAs of one grid (cluster launch control) ---------------
+// Ask the hardware to cancel the launch of a CTA of this grid that has not started yet; the
+// 16-byte response lands in shared memory and completes 16 bytes of transaction on `bar`.
+// After a response that reports failure, no further request may be made.
+__device__ __forceinline__ void work_request(uint32_t resp, uint32_t bar)
+{
+    asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+                 ::"r"(resp), "r"(bar)
+                 : "memory");
+}
+// Decode a response: true and the cancelled CTA's x index, or false (no CTA left to take).
+__device__ __forceinline__ bool work_response(uint32_t resp, uint32_t &ctaid_x)
+{
+    uint32_t ok, x;
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+                 "ld.shared.b128 r, [%2];\n\t"
+                 "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t"
+                 "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+                 : "=r"(ok), "=r"(x)
+                 : "r"(resp)
+                 : "memory");
+    ctaid_x = x;
+    return ok != 0;
+}
+
 // ---- bulk copies (TMA engine) --------------------------------------------------------
 // 1-D bulk copy global -> shared, completing `bytes` of transaction on an mbarrier.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)

@@ -13,7 +13,8 @@ constexpr int kMaxTemporalGroup = 4;   // heads per work item = consumer warps p
 constexpr int kMaxChunk = 8;           // queries per (token, head): the chunk length limit
 
 struct TemporalParams {
-    __nv_bfloat16 *out;                 // [B][n][HW][H][D]
+    __nv_bfloat16 *out;                 // [B][HW][n][H][D]
+    const uint8_t *rk, *rv;             // this layer's K and V rings [B][HW][H][Pmax][D]
     int B, HW, H, D;
     int n;          // chunk frames in this call (queries per token-head)
     int Pk;         // queued frames
@@ -25,10 +26,10 @@ struct TemporalParams {
     float scale_log2;         // log2(e) / sqrt(D)
 };
 
-// 5-D views (head dim, frame, head, token, video) of the chunk tensors and of one
-// layer's K and V rings; boxes of D x 16 frames x G heads (D x 8 x G for q).
+// 5-D views (head dim, frame, head, token, video) of the chunk tensors; boxes of
+// D x 16 frames x G heads (D x 8 x G for q).  The rings are read with 1-D bulk copies.
 struct TemporalMaps {
-    CUtensorMap q, k, v, rk, rv;
+    CUtensorMap q, k, v;
 };
 
 constexpr int kMaxRingSlots = 16 * 32;   // the ring-box mask has 32 bits
@@ -45,9 +46,11 @@ struct CacheWriteLayer {
 
 struct CacheWriteParams {
     CacheWriteLayer layer[kMaxLayersPerWrite];
-    uint4 *tbuf;            // temporal cache base [N_L][2][B][HW][Pmax][C] (token-major ring)
+    uint4 *tbuf;            // temporal cache base [N_L][2][B][HW][H][Pmax][D] (token-major, head-major ring)
     uint4 *sbuf;            // spatial cache base  [N_L][2][P'][B][HW][C]
     long long row_vec;      // 16-byte vectors per row of C = H*D elements
+    int head_vec;           // 16-byte vectors per head row of D elements
+    int heads;
     long long tokens;       // B * HW
     int hw;
     int layer0;             // absolute index of layer[0]

@@ -4,8 +4,9 @@
 // one clean forward pass computes its K/V, which join the temporal queue (FIFO, at most
 // Pmax frames) and replace the one-chunk spatial cache.  This kernel is the data movement
 // of that step for every layer at once: a bit-exact copy, 16 bytes per access.  The ring
-// is token-major (each token's Pmax slots are contiguous), so a temporal write moves the
-// chunk's n rows of every token into that token's slots.
+// is token-major and head-major within a token ([B][HW][H][Pmax][D]: one head's Pmax slots
+// are contiguous), so a temporal write moves each (token, frame, head) row of D elements of
+// the chunk into that head's slot.
 #include <cstdint>
 
 #include "ca2_device.cuh"
@@ -30,7 +31,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 }  // namespace
 
 // blockIdx.y = (layer, tensor): tensor 0/1 = temporal K/V, 2/3 = spatial K/V.
-//   temporal: chunk [B][HW][n][C] -> ring [B][HW][Pmax][C]; row (token, j) -> slot (slot0 + j) mod Pmax
+//   temporal: chunk [B][HW][n][H][D] -> ring [B][HW][H][Pmax][D]; (token, j, h) -> slot (slot0 + j) mod Pmax
 //   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
@@ -66,8 +67,10 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
                 const int j = (int)(row - tok * p.n);
                 int slot = p.slot0 + j;
                 if (slot >= p.p_max) slot -= p.p_max;
+                const int h = (int)(off / p.head_vec);
+                const long long dv = off - (long long)h * p.head_vec;
                 so[i] = e;
-                dof[i] = (tok * p.p_max + slot) * rv + off;
+                dof[i] = ((tok * p.heads + h) * p.p_max + slot) * p.head_vec + dv;
             } else {
                 // row = jsp * tokens + (b * HW + s); source frame n - n_sp + jsp of video b
                 const long long jsp = row / p.tokens;

@@ -9,29 +9,34 @@
 // ring read one contiguous run.  Only the chunk's own keys carry the causal mask.
 //
 // Design (HBM-bound: each cached K/V byte is read once per call):
-//   * Temporal tensors are token-major: the chunk is [B][HW][n][H][D] and the ring
-//     [B][HW][Pmax][H][D], so one token's whole history is one contiguous run (41 x 2304 B
-//     at the Open-Sora shape) and the reads keep DRAM pages open.
-//   * Work item = (video b, token s, group of G heads).  Tensor maps view the ring and
-//     the chunk tensors as 5-D (head dim, frame, head, token, video) -- dimension order
-//     chosen so that one TMA box (D x 16 frames x G heads) lands in shared memory as
-//     [head][frame][D]: each head's 16 key rows are consecutive 2*D-byte rows (an odd
-//     number of 16-byte units for D = 72, so ldmatrix is bank-conflict free), and one
-//     TMA operation moves 16 frames x G heads (9.2 KB at G = 4, D = 72).
-//   * Stage 0 is the chunk's own 16-frame box (frames past n are zero-filled by the TMA
-//     unit), then the ring in 16-slot boxes (slots past Pmax zero-filled).  Stage 0
+//   * Temporal tensors are token-major: the chunk is [B][HW][n][H][D]; the ring is
+//     [B][HW][H][Pmax][D], head-major within a token, so one (token, head) history is one
+//     contiguous run (41 x 144 B at the Open-Sora shape).
+//   * Work item = (video b, token s, group of G heads).  A stage holds 16 key frames of
+//     the G heads, in shared memory as [head][frame][D]: each head's 16 key rows are
+//     consecutive 2*D-byte rows (an odd number of 16-byte units for D = 72, so ldmatrix is
+//     bank-conflict free).
+//   * Stage 0 is the chunk's own 16 frames, one TMA box per tensor viewed 5-D (head dim,
+//     frame, head, token, video); frames past n are zero-filled by the TMA unit.  Stage 0
 //     holds chunk frame 0, which every query sees, so the running max is finite from the
-//     first stage on.  Ring boxes with no queued slot are skipped (host-computed mask).
-//   * Persistent CTAs: one producer warp keeps NS stages of K and V in flight on
-//     mbarriers and runs ahead across items; G consumer warps (one head each) compute.
+//     first stage on.  Then the ring in 16-slot groups: per head one bulk copy of the
+//     group's consecutive slots (2304 B for a full group; contiguous copies of this size
+//     stream at the HBM rate, where boxes of 144-byte rows measured well below it).
+//     Groups with no queued slot are skipped (host-computed mask).
+//   * Work distribution: one CTA per work item in the grid; a resident CTA finishes its
+//     own item and then takes over the items of CTAs that have not started yet (cluster
+//     launch control), so every SM stays busy to the end whatever its share of items.
+//     One producer warp keeps NS stages of K and V in flight on mbarriers and runs ahead
+//     across items; G consumer warps (one head each) compute.
 //   * Per head the contraction is tiny (8 queries x 16 keys per stage x D), so both
 //     products use mma.sync on registers: S^T = K Q^T (keys on M, the 8 queries on N),
 //     then O^T += V^T P^T.  Each lane owns the same two query columns in both
 //     accumulators, so the online-softmax rescale is lane-local; movmatrix turns P^T
 //     into the B operand and O^T back into rows for the stores.
-//   * Ring slots that hold no queued frame (before the queue is full) are masked; their
-//     V rows are zeroed in shared memory before use, so stale cache contents (whatever
-//     bits the caller's buffer held) never reach the accumulator.
+//   * Ring rows that hold no queued frame (slots not yet queued, and rows past Pmax that
+//     the copy did not write) are masked; their V rows are zeroed in shared memory before
+//     use, so stale bits (of the caller's buffer or of an earlier stage) never reach the
+//     accumulator.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -43,7 +48,7 @@ namespace ca2 {
 namespace {
 
 constexpr int kStages = 5;       // K+V stages in flight per CTA
-constexpr int kKeys = 16;        // key frames per stage (one TMA box)
+constexpr int kKeys = 16;        // key frames per stage
 constexpr int kQ = 8;            // queries per (token, head): the mma N extent
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
@@ -112,7 +117,7 @@ struct Layout {
     uint32_t kv_box;        // bytes of one K (or V) box: G heads x 16 frames x D
     uint32_t stage_bytes;   // K box then V box
     uint32_t q_box;         // G heads x 8 frames x D
-    uint32_t q_off, bar_off, total;
+    uint32_t q_off, bar_off, misc_off, total;
 };
 
 __host__ __device__ inline Layout make_layout(int G, int D)
@@ -123,7 +128,9 @@ __host__ __device__ inline Layout make_layout(int G, int D)
     L.q_box = (uint32_t)(G * kQ * D * 2);
     L.q_off = kStages * L.stage_bytes;
     L.bar_off = (L.q_off + 2u * L.q_box + 7u) & ~7u;
-    L.total = L.bar_off + 8u * (2 * kStages + 4) + 16u;
+    // after the barriers: the 16-byte work-request response, the abort flag, two item ids
+    L.misc_off = (L.bar_off + 8u * (2 * kStages + 5) + 15u) & ~15u;
+    L.total = L.misc_off + 32u;
     return L;
 }
 
@@ -132,8 +139,7 @@ __host__ __device__ inline Layout make_layout(int G, int D)
 template <int DT>
 __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
     k_temporal_causal(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_rk,
-                      const __grid_constant__ CUtensorMap tm_rv, const TemporalParams p)
+                      const __grid_constant__ CUtensorMap tm_v, const TemporalParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
@@ -147,7 +153,10 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
     auto empty_bar = [&](int i) { return bar0 + 8u * (kStages + i); };
     auto qfull_bar = [&](int i) { return bar0 + 8u * (2 * kStages + i); };
     auto qempty_bar = [&](int i) { return bar0 + 8u * (2 * kStages + 2 + i); };
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.bar_off + 8u * (2 * kStages + 4));
+    auto work_bar = [&]() { return bar0 + 8u * (2 * kStages + 4); };
+    const uint32_t work_resp = sbase + L.misc_off;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc_off + 16u);
+    volatile int *item_ids = reinterpret_cast<volatile int *>(smem + L.misc_off + 20u);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -158,6 +167,7 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
             mbar_init(qfull_bar(i), 1);
             mbar_init(qempty_bar(i), G);
         }
+        mbar_init(work_bar(), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -170,46 +180,105 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
 
     if (warp == G) {
         // ------------------------------ producer ------------------------------------
+        // The whole warp runs the loop (warp-uniform waits); lane 0 issues the TMA boxes and
+        // the work requests, and the ring copies of a stage go out in one warp instruction,
+        // lane i < 2G issuing one head's K (i < G) or V run: a single issuing thread was
+        // measured at ~150 cycles per bulk copy.
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            prefetch_tmap(&tm_rk);
-            prefetch_tmap(&tm_rv);
-            int stage = 0, li = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++li) {
-                const int hg = it % groups;
-                const int s = (it / groups) % p.HW;
-                const int b = it / (groups * p.HW);
-                const int qs = li & 1;
-                if (li >= 2 && !mbar_wait(qempty_bar(qs), ((li - 2) >> 1) & 1, 101, abort_flag)) { ok = false; break; }
+        }
+        // Work items: this CTA's own index first, then items of CTAs of the grid that
+        // have not started yet, taken over through cluster launch control until none is
+        // left; every SM stays busy until the last items, whatever their count per SM.
+        int stage = 0, li = 0;
+        int requests = 0;           // work requests made (phases of work_bar)
+        bool can_take = true;       // no request has failed yet
+        bool pending = false;       // a request whose response has not been read
+        bool ok = true;
+        int it = blockIdx.x;
+        while (ok && it >= 0 && it < p.n_items) {
+            const int hg = it % groups;
+            const int s = (it / groups) % p.HW;
+            const int b = it / (groups * p.HW);
+            const int qs = li & 1;
+            // ask for the next item now; the answer comes back while this one loads
+            if (can_take) {
+                if (lane == 0) {
+                    mbar_expect_tx(work_bar(), 16u);
+                    work_request(work_resp, work_bar());
+                }
+                pending = true;
+            }
+            if (li >= 2 && !warp_wait(qempty_bar(qs), ((li - 2) >> 1) & 1, 101, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
+                item_ids[qs] = it;
                 mbar_expect_tx(qfull_bar(qs), L.q_box);
                 tma_load_5d(sbase + L.q_off + (uint32_t)qs * L.q_box, &tm_q, 0, 0, hg * G, s, b, qfull_bar(qs));
-                uint32_t mask = p.ring_box_mask;
-                for (int st = 0; st < n_stages; ++st, ++stage) {
-                    const int slot = stage % kStages;
-                    if (stage >= kStages &&
-                        !mbar_wait(empty_bar(slot), ((stage / kStages) - 1) & 1, 102, abort_flag)) { ok = false; break; }
-                    const uint32_t dst = sbase + (uint32_t)slot * L.stage_bytes;
-                    mbar_expect_tx(full_bar(slot), L.stage_bytes);
-                    if (st == 0) {
+            }
+            ++li;
+            uint32_t mask = p.ring_box_mask;
+            for (int st = 0; st < n_stages; ++st, ++stage) {
+                const int slot = stage % kStages;
+                if (stage >= kStages &&
+                    !warp_wait(empty_bar(slot), ((stage / kStages) - 1) & 1, 102, abort_flag)) { ok = false; break; }
+                const uint32_t dst = sbase + (uint32_t)slot * L.stage_bytes;
+                if (st == 0) {
+                    if (lane == 0) {
+                        mbar_expect_tx(full_bar(slot), L.stage_bytes);
                         tma_load_5d(dst, &tm_k, 0, 0, hg * G, s, b, full_bar(slot));
                         tma_load_5d(dst + L.kv_box, &tm_v, 0, 0, hg * G, s, b, full_bar(slot));
-                    } else {
-                        const int box = __ffs(mask) - 1;
-                        mask &= mask - 1;
-                        tma_load_5d(dst, &tm_rk, 0, box * kKeys, hg * G, s, b, full_bar(slot));
-                        tma_load_5d(dst + L.kv_box, &tm_rv, 0, box * kKeys, hg * G, s, b, full_bar(slot));
+                    }
+                } else {
+                    // ring slots [16 box, 16 box + ns): one contiguous run of ns rows per
+                    // head and tensor (the ring is head-major within a token)
+                    const int box = __ffs(mask) - 1;
+                    mask &= mask - 1;
+                    const int s0 = box * kKeys;
+                    const int ns = min(kKeys, p.Pmax - s0);
+                    const uint32_t run = (uint32_t)(ns * D * 2);
+                    if (lane == 0) mbar_expect_tx(full_bar(slot), 2u * (uint32_t)G * run);
+                    __syncwarp();
+                    if (lane < 2 * G) {
+                        const int w = lane % G;
+                        const int kv = lane / G;
+                        const size_t off = ((((size_t)b * p.HW + (size_t)s) * (size_t)p.H + (size_t)(hg * G + w)) *
+                                                (size_t)p.Pmax + (size_t)s0) * ((size_t)D * 2u);
+                        bulk_g2s(dst + (uint32_t)kv * L.kv_box + (uint32_t)(w * kKeys * D * 2),
+                                 (kv ? p.rv : p.rk) + off, run, full_bar(slot));
                     }
                 }
             }
+            if (!ok) break;
+            int next = -1;
+            if (pending) {
+                if (!warp_wait(work_bar(), requests & 1, 105, abort_flag)) { ok = false; break; }
+                ++requests;
+                pending = false;
+                uint32_t x;
+                if (work_response(work_resp, x)) next = (int)x;
+                else can_take = false;
+            }
+            it = next;
+        }
+        if (lane == 0) {
+            // no further item: a sentinel in the next Q slot ends the consumers' loop
+            if (ok) {
+                const int qs = li & 1;
+                if (li < 2 || mbar_wait(qempty_bar(qs), ((li - 2) >> 1) & 1, 101, abort_flag)) {
+                    item_ids[qs] = -1;
+                    mbar_arrive(qfull_bar(qs));
+                }
+            }
+            // an unanswered request still writes shared memory: wait for it (bounded)
+            if (pending) mbar_wait(work_bar(), requests & 1, 0, nullptr, 2000000ull);
             // wind-down after an abort: let the loads still in flight land before exiting
             // (each slot's last use is the most recent phase of its barrier)
             if (!ok) {
                 for (int k = stage - 1; k >= 0 && k >= stage - kStages; --k)
                     mbar_wait(full_bar(k % kStages), (k / kStages) & 1, 0, nullptr, 2000000ull);
-                for (int k = li; k >= 0 && k >= li - 1; --k)
+                for (int k = li - 1; k >= 0 && k >= li - 2; --k)
                     mbar_wait(qfull_bar(k & 1), (k >> 1) & 1, 0, nullptr, 2000000ull);
             }
         }
@@ -222,13 +291,15 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
         const int q0 = 2 * (lane & 3);        // this lane's two query columns: q0, q0 + 1
         const int krow = lane >> 2;            // this lane's key rows in a stage: krow, krow + 8
         const float neg_inf = __int_as_float(0xff800000);
-        int stage = 0, li = 0;
-        for (int it = blockIdx.x; it < p.n_items; it += gridDim.x, ++li) {
+        int stage = 0;
+        for (int li = 0;; ++li) {
+            const int qs = li & 1;
+            if (!warp_wait(qfull_bar(qs), (li >> 1) & 1, 103, abort_flag)) break;
+            const int it = item_ids[qs];      // written before the Q slot's barrier arrive
+            if (it < 0) break;
             const int hg = it % groups;
             const int s = (it / groups) % p.HW;
             const int b = it / (groups * p.HW);
-            const int qs = li & 1;
-            if (!warp_wait(qfull_bar(qs), (li >> 1) & 1, 103, abort_flag)) break;
 
             // Q as the B operand (col-major K x N = dims x queries == Q rows [query][dim])
             uint32_t qb[DT][2];
@@ -276,11 +347,12 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         const bool v = sl < p.Pmax && age < p.Pk;
                         vis[hr][0] = vis[hr][1] = v;
                     }
-                    // slots inside the ring that hold no queued frame: zero their V rows
+                    // rows that hold no queued frame (stale slots, and rows past Pmax that the
+                    // copy did not write): zero their V rows
                     const int sl = box * kKeys + (lane & 15);
                     int age = sl - p.head;
                     if (age < 0) age += p.Pmax;
-                    zero_v = sl < p.Pmax && age >= p.Pk;
+                    zero_v = !(sl < p.Pmax && age < p.Pk);
                 }
                 if (!warp_wait(full_bar(slot), (stage / kStages) & 1, 104, abort_flag)) { ok = false; break; }
                 const uint32_t kbase = sbase + (uint32_t)slot * L.stage_bytes + head_kv;
@@ -407,7 +479,7 @@ static cudaError_t launch_dt(const TemporalMaps &m, const TemporalParams &p, int
         if (e != cudaSuccess) return e;
         configured_for = dev;
     }
-    k_temporal_causal<DT><<<grid, 32 * (p.G + 1), smem, stream>>>(m.q, m.k, m.v, m.rk, m.rv, p);
+    k_temporal_causal<DT><<<grid, 32 * (p.G + 1), smem, stream>>>(m.q, m.k, m.v, p);
     return cudaGetLastError();
 }
 

@@ -28,8 +28,9 @@
  *   - A handle is not thread-safe.
  *
  * Cache memory layout (both buffers caller-allocated, sizes from ca2_cache_bytes):
- *   temporal: [N_L][2][B][HW][Pmax][H][D]   (index 0 = K ring, 1 = V ring; token-major:
- *                                            a token's Pmax slots are contiguous)
+ *   temporal: [N_L][2][B][HW][H][Pmax][D]   (index 0 = K ring, 1 = V ring; token-major and
+ *                                            head-major within a token: one head's Pmax
+ *                                            slots are contiguous)
  *   spatial : [N_L][2][P'][B][HW][H][D]
  * The i-th oldest queued frame (i = 0 .. count-1) is in ring slot (head + i) mod Pmax;
  * spatial slot j (j < sp_count) holds the j-th of the last sp_count frames written,

@@ -127,8 +127,8 @@ class Loop:
             rv = to_bits(self.cache.ring(L, 1))
             for g in ring.queue:
                 slot = ring.slot_of(g)
-                assert np.array_equal(rk[:, :, slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
-                assert np.array_equal(rv[:, :, slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rk[:, :, :, slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rv[:, :, :, slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
             if self.wl.p_spatial:
                 sk = to_bits(self.cache.spatial(L, 0))
                 sv = to_bits(self.cache.spatial(L, 1))
