@@ -218,6 +218,29 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x on the FMA pipe, for x <= 0 (a score minus the running max, log2 units): x = n + f
+// with n the nearest integer (by the 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5];
+// 2^f by a degree-3 polynomial fitted here for minimal relative error (max 7.5e-5, well
+// under bf16's 3.9e-3 rounding step); 2^n added to the exponent bits.  Inputs below -127
+// are clamped (the result is then below 2^-126, zero for the bf16 probabilities).
+__device__ __forceinline__ float ex2_fma(float x)
+{
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;
+    const float n = t - 12582912.f;
+    const float f = x - n;
+    const float q = fmaf(fmaf(fmaf(0.05517196f, f, 0.24261114f), f, 0.69326091f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(q) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
 // 32 lanes x 128 consecutive 32-bit columns (two x64 loads, one wait).
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
 {
@@ -588,15 +611,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
 #pragma unroll
             for (int i = 0; i < 8; ++i) m8[i] = neg_inf;
             if (valid >= kKeys) {
+                // 8 independent chains, two scores per three-input max
 #pragma unroll
-                for (int i = 0; i < kKeys; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
+                for (int i = 0; i < kKeys; i += 16)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        m8[c] = fmax3(m8[c], __uint_as_float(sr[i + c]), __uint_as_float(sr[i + 8 + c]));
             } else {
 #pragma unroll
                 for (int i = 0; i < kKeys; ++i)
                     if (i < valid) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
             }
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale;
+            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * scale;
             float alpha = 1.f;
             const bool upd = mx > m_used + kLazyRescale;
             if (upd) {

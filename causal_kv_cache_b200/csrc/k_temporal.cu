@@ -203,14 +203,6 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
             const int s = (it / groups) % p.HW;
             const int b = it / (groups * p.HW);
             const int qs = li & 1;
-            // ask for the next item now; the answer comes back while this one loads
-            if (can_take) {
-                if (lane == 0) {
-                    mbar_expect_tx(work_bar(), 16u);
-                    work_request(work_resp, work_bar());
-                }
-                pending = true;
-            }
             if (li >= 2 && !warp_wait(qempty_bar(qs), ((li - 2) >> 1) & 1, 101, abort_flag)) { ok = false; break; }
             if (lane == 0) {
                 item_ids[qs] = it;
@@ -251,7 +243,19 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                 }
             }
             if (!ok) break;
+            // claim the next item only once a ring slot is free for its first stage: a claim
+            // made earlier would reserve it long before this CTA can start on it, and the
+            // CTAs holding one more item at the end of the list set the tail
             int next = -1;
+            if (can_take) {
+                if (stage >= kStages &&
+                    !warp_wait(empty_bar(stage % kStages), ((stage / kStages) - 1) & 1, 102, abort_flag)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_expect_tx(work_bar(), 16u);
+                    work_request(work_resp, work_bar());
+                }
+                pending = true;
+            }
             if (pending) {
                 if (!warp_wait(work_bar(), requests & 1, 105, abort_flag)) { ok = false; break; }
                 ++requests;
