@@ -99,6 +99,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int sit
     return __all_sync(0xffffffffu, ok);
 }
 
+// ---- programmatic dependent launch ------------------------------------------------------
+// The attention kernels are launched so that the next kernel on the stream may start while
+// this one drains.  Each kernel does its set-up (barriers, TMEM, tensor-map prefetch), then
+// every thread waits for the previous kernel on the stream to complete (its memory visible)
+// before touching global memory, and only then lets its own dependent start: so a kernel's
+// set-up never overlaps anything but its immediate predecessor's last CTAs.
+__device__ __forceinline__ void wait_previous_kernel() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_kernel() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- work stealing between CTAs of one grid (cluster launch control) ---------------
 // Ask the hardware to cancel the launch of a CTA of this grid that has not started yet; the
 // 16-byte response lands in shared memory and completes 16 bytes of transaction on `bar`.

@@ -226,21 +226,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c)
     return r;
 }
 
-// 2^x on the FMA pipe, for x <= 0 (a score minus the running max, log2 units): x = n + f
-// with n the nearest integer (by the 1.5 * 2^23 rounding constant) and f in [-0.5, 0.5];
-// 2^f by a degree-3 polynomial fitted here for minimal relative error (max 7.5e-5, well
-// under bf16's 3.9e-3 rounding step); 2^n added to the exponent bits.  Inputs below -127
-// are clamped (the result is then below 2^-126, zero for the bf16 probabilities).
-__device__ __forceinline__ float ex2_fma(float x)
-{
-    x = fmaxf(x, -127.f);
-    const float t = x + 12582912.f;
-    const float n = t - 12582912.f;
-    const float f = x - n;
-    const float q = fmaf(fmaf(fmaf(0.05517196f, f, 0.24261114f), f, 0.69326091f), f, 0.99992806f);
-    return __int_as_float(__float_as_int(q) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // 32 lanes x 128 consecutive 32-bit columns (two x64 loads, one wait).
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
 {
@@ -410,13 +395,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         for (int i = 0; i < kChunks; ++i) mbar_init(bar(B_PFREE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
-        // the first loads go out before TMEM allocation and the CTA-wide sync
         prefetch_tmap(&tm.q);
         prefetch_tmap(&tm.k);
         prefetch_tmap(&tm.v);
         prefetch_tmap(&tm.sk);
         prefetch_tmap(&tm.sv);
         prefetch_tmap(&tm.o);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32((const void *)tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // the previous kernel on the stream has completed: inputs may now be read
+    wait_previous_kernel();
+    allow_next_kernel();
+    if (threadIdx.x == 0) {
         mbar_expect_tx(bar(B_QFULL), 2 * tile_bytes(NKD));
         load_tile(sb + L.q0, &tm.q, row0, b * p.n + f, bar(B_QFULL));
         load_tile(sb + L.q0 + TB, &tm.q, row0 + kRows, b * p.n + f, bar(B_QFULL));
@@ -430,13 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             load_tile(sb + L.v0, mv, r, fr, bar(B_VFULL));
         }
     }
-    if (warp == 1) {
-        tmem_alloc(smem_u32((const void *)tmem_slot), kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // When D is not a multiple of 32 the P V product has padding columns D..DP-1; column D
     // of every V tile is set to 1.0 so that the tensor core also accumulates the row sum
@@ -765,8 +754,7 @@ static cudaError_t launch_nkd(const SpatialMaps &m, const SpatialParams &p, cuda
         configured_for = dev;
     }
     const unsigned grid = (unsigned)(p.B * p.n * p.H * p.q_pairs);
-    k_spatial_prefix<NKD><<<grid, kThreads, smem, stream>>>(m, p);
-    return cudaGetLastError();
+    return launch_chained(k_spatial_prefix<NKD>, dim3(grid), dim3(kThreads), smem, stream, m, p);
 }
 
 cudaError_t launch_spatial(const SpatialMaps &m, const SpatialParams &p, cudaStream_t stream)

@@ -170,8 +170,14 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
         mbar_init(work_bar(), 1);
         *abort_flag = 0;
         fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
     }
     __syncthreads();
+    // the previous kernel on the stream has completed: inputs may now be read
+    wait_previous_kernel();
+    allow_next_kernel();
 
     const int groups = p.H / G;
     // stage list: stage 0 = the chunk's frames, then the ring boxes whose bit is set
@@ -184,11 +190,6 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
         // the work requests, and the ring copies of a stage go out in one warp instruction,
         // lane i < 2G issuing one head's K (i < G) or V run: a single issuing thread was
         // measured at ~150 cycles per bulk copy.
-        if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-        }
         // Work items: this CTA's own index first, then items of CTAs of the grid that
         // have not started yet, taken over through cluster launch control until none is
         // left; every SM stays busy until the last items, whatever their count per SM.
@@ -483,8 +484,7 @@ static cudaError_t launch_dt(const TemporalMaps &m, const TemporalParams &p, int
         if (e != cudaSuccess) return e;
         configured_for = dev;
     }
-    k_temporal_causal<DT><<<grid, 32 * (p.G + 1), smem, stream>>>(m.q, m.k, m.v, p);
-    return cudaGetLastError();
+    return launch_chained(k_temporal_causal<DT>, dim3(grid), dim3(32 * (p.G + 1)), smem, stream, m.q, m.k, m.v, p);
 }
 
 cudaError_t launch_temporal(const TemporalMaps &m, const TemporalParams &p, int grid, cudaStream_t stream)
