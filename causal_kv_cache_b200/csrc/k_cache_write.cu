@@ -35,10 +35,6 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 //   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
-    // the previous kernel on the stream (the last attention pass reads the cache) has
-    // completed before any cache byte is written.  The next kernel is not let in early: its
-    // CTAs would hold whole SMs, waiting, that this grid's many short CTAs still need.
-    wait_previous_kernel();
     const int li = blockIdx.y >> 2;
     const int tensor = blockIdx.y & 3;
     const CacheWriteLayer &Ly = p.layer[li];
@@ -99,7 +95,10 @@ cudaError_t launch_cache_write(const CacheWriteParams &p, cudaStream_t stream)
     const long long most = t_total > s_total ? t_total : s_total;
     dim3 grid((unsigned)((most + per_block - 1) / per_block), (unsigned)(p.n_layers * 4));
     if (grid.x == 0 || grid.y == 0) return cudaSuccess;
-    return launch_chained(k_cache_write, grid, dim3(kThreads), 0, stream, p);
+    // a plain launch: it starts only after the previous kernel on the stream (the last
+    // attention pass reads the cache) has completed
+    k_cache_write<<<grid, kThreads, 0, stream>>>(p);
+    return cudaGetLastError();
 }
 
 // ---- bounded-wait self test -------------------------------------------------------------
