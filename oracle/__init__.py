@@ -18,6 +18,10 @@ What it holds (all plain definitions, fp64 for floating point, integers exact):
   every write (papernotes page, 关键设计 4 and 5).
 * ``tpe_indices``    -- cyclic temporal-position indices (papernotes page, 关键设计 4,
   "Cyclic-TPEs"): index of global frame g is (offset + g) mod N_tpe.
+* ``tpe_add``        -- the chunk input plus each frame's TPE row at its cyclic index,
+  added to every token's channel vector (the reading taken: the embedding is added to the
+  temporal branch's input, as the pages' Open-Sora backbone does).  Sum in float32, one
+  rounding to bf16 (nearest, ties to even), the precision the kernel computes in.
 * ``cache_bytes``    -- bytes of the shared KV cache (K and V, 2-byte elements,
   Pmax temporal frames plus P' spatial frames per layer).
 
@@ -171,6 +175,35 @@ def tpe_indices(first_global_frame: int, offset: int, n: int, n_tpe: int) -> Lis
     if n_tpe <= 0:
         raise ValueError("n_tpe must be positive")
     return [(offset + first_global_frame + c) % n_tpe for c in range(n)]
+
+
+def bf16_round_bits(x: np.ndarray) -> np.ndarray:
+    """float32 values -> bfloat16 bits, rounded to nearest with ties to even (IEEE)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = (u & 0x7FFFFFFF) > 0x7F800000
+    r[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)    # keep NaN a (quiet) NaN
+    return r
+
+
+def tpe_add(x: np.ndarray, table: np.ndarray, first_global_frame: int, offset: int) -> np.ndarray:
+    """x + TPE for one chunk, token-major: x [B][HW][n][C] bf16 bits, table [N_tpe][C] bf16 bits.
+
+    Frame f of the chunk (global frame first_global_frame + f) gets row
+    tpe_indices(first_global_frame, offset, n, N_tpe)[f] of the table added to every token's
+    C-vector ("Ca2-VDM" papernotes page, 关键设计 4 "Cyclic-TPEs").  Each element is the
+    float32 sum of the two bf16 values rounded once to bf16 (ties to even).
+    """
+    x = _u16(x)
+    table = _u16(table)
+    n, C = x.shape[2], x.shape[3]
+    if table.ndim != 2 or table.shape[1] != C:
+        raise ValueError("table must be [N_tpe][C] with the chunk's C")
+    idx = tpe_indices(first_global_frame, offset, n, table.shape[0])
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    tf = (table.astype(np.uint32) << 16).view(np.float32)[idx]          # [n][C]
+    return bf16_round_bits(xf + tf[None, None, :, :])
 
 
 def cache_bytes(n_layers: int, batch: int, hw: int, heads: int, head_dim: int,

@@ -167,3 +167,34 @@ def test_planted_mistake_is_caught(tmp_path, name, old, new, occ):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, "planted mistake %r passed every pin" % name
+
+
+def _bits(vals):
+    return np.asarray(vals, dtype=np.float32).view(np.uint32).__rshift__(16).astype(np.uint16)
+
+
+def test_tpe_add_zero_table_is_identity():
+    rng = np.random.default_rng(4)
+    x = rng.integers(0, 0x7F00, size=(2, 5, 3, 16), dtype=np.uint16)
+    table = np.zeros((7, 16), dtype=np.uint16)
+    assert np.array_equal(oracle.tpe_add(x, table, 5, 2), x)
+
+
+def test_tpe_add_on_zero_input_gathers_cyclic_rows():
+    """x = 0: the result is the table rows at (offset + g0 + f) mod N_tpe, wrap included."""
+    n_tpe, C = 7, 16
+    table = _bits(np.arange(n_tpe * C, dtype=np.float32).reshape(n_tpe, C) + 1.0)   # exact in bf16
+    x = np.zeros((1, 3, 4, C), dtype=np.uint16)
+    out = oracle.tpe_add(x, table, 5, 3)          # frames 5..8, offset 3 -> rows 1, 2, 3, 4
+    for f, row in enumerate([1, 2, 3, 4]):
+        assert np.array_equal(out[0, :, f], np.broadcast_to(table[row], (3, C)))
+    out = oracle.tpe_add(x, table, 12, 0)         # rows 5, 6, 0, 1
+    assert [int(np.argmax(np.all(out[0, 0, f] == table, axis=1))) for f in range(4)] == [5, 6, 0, 1]
+
+
+def test_tpe_add_rounds_ties_to_even():
+    """1 + 2^-8 lies halfway between 1 and 1 + 2^-7 in bf16: ties go to the even mantissa."""
+    table = _bits([[2.0 ** -8, 2.0 ** -8, 3.0 * 2.0 ** -9]])
+    x = _bits([1.0, 1.0078125, 1.0]).reshape(1, 1, 1, 3)
+    out = oracle.tpe_add(x, table, 0, 0)
+    assert out.reshape(-1).tolist() == [0x3F80, 0x3F82, 0x3F81]   # 1.0, 1.015625, 1.0078125
