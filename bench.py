@@ -312,12 +312,34 @@ def run_ca2(args):
     tokens_per_step = (T + 1) * NL * B * l * HW
     value = whole_job_rate(tokens_per_step, args.steps, world, ms)
 
+    # ---- cyclic TPE add (a next-row kernel, timed on its own, outside the step) ----
+    # 28 launches (one per block's temporal input) in a CUDA graph, replayed 5 times
+    tpe_table = (torch.randn((cache.tpe_len, H, D), generator=g, device=dev) * 0.7).to(torch.bfloat16)
+    tpe_out = [torch.empty((B, HW, l, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    gt = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        gt.capture_begin()
+        for L in range(NL):
+            ca2.ca2_tpe_add(h, g0[0], 0, tpe_table, P[L]["tq"], tpe_out[L], l, cap_sp)
+        gt.capture_end()
+    gt.replay()
+    torch.cuda.synchronize()
+    ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ta.record(stream)
+    for _ in range(5):
+        gt.replay()
+    tb.record(stream)
+    torch.cuda.synchronize()
+    avg_tpe = ta.elapsed_time(tb) / 1e3 / (5 * NL)
+    del gt
+
     # ---- roofline of each kernel ----
     pk, pk_kind = peaks()
     t_bytes = (2 * PM + 4 * l) * frame_bytes                       # cache K,V + chunk Q,K,V + O
     s_flops_den = 4 * D * HW * (1 + PS) * HW * l * H * B           # denoising mode (P' prefix frames)
     s_flops_self = 4 * D * HW * HW * l * H * B                     # self-repeat mode (own frame once)
     w_bytes = 2 * NL * (2 * l + 2 * PS) * frame_bytes              # read + write of K,V (temporal, spatial)
+    tpe_bytes = 2 * l * frame_bytes + l * H * D * 2                 # chunk read + write, n table rows
     avg_t = statistics.mean(tp_ms) / 1e3
     avg_sd = statistics.mean(sp_den) / 1e3
     avg_ss = statistics.mean(sp_self) / 1e3
@@ -331,6 +353,9 @@ def run_ca2(args):
                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "flops_per_launch": s_flops_self},
         "cache_write": {"bound": "hbm", "us": avg_w * 1e6, "achieved": w_bytes / avg_w / 1e9,
                         "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": w_bytes},
+        "tpe_add": {"bound": "hbm", "us": avg_tpe * 1e6, "achieved": tpe_bytes / avg_tpe / 1e9,
+                    "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": tpe_bytes,
+                    "note": "timed apart from the step: 28 launches in a graph, replayed 5 times"},
     }
     for k in kernels.values():
         k["frac"] = k["achieved"] / k["peak"]

@@ -18,7 +18,7 @@ from typing import List, Optional, Sequence, Tuple
 __all__ = [
     "Ca2Error", "ca2_config", "load_library", "LIBRARY_PATH",
     "ca2_cache_bytes", "ca2_cache_init", "ca2_cache_destroy", "ca2_cache_evict",
-    "ca2_cache_write", "ca2_temporal_attn", "ca2_spatial_prefix_attn", "ca2_tpe_indices",
+    "ca2_cache_write", "ca2_temporal_attn", "ca2_spatial_prefix_attn", "ca2_tpe_indices", "ca2_tpe_add",
     "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string",
     "ca2_last_error_string",
     "KVCache", "STATUS",
@@ -79,6 +79,7 @@ def load_library(path: Optional[str] = None):
         "ca2_temporal_attn": ([vp, i, vp, vp, vp, vp, i, vp], i),
         "ca2_spatial_prefix_attn": ([vp, i, vp, vp, vp, vp, i, i, vp], i),
         "ca2_tpe_indices": ([vp, ll, i, i, ctypes.POINTER(ctypes.c_int)], i),
+        "ca2_tpe_add": ([vp, ll, i, vp, vp, vp, i, vp], i),
         "ca2_cache_state": ([vp, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(ll)], i),
         "ca2_device_status": ([], i),
         "ca2_selftest_timeout": ([i, vp], i),
@@ -190,6 +191,12 @@ def ca2_spatial_prefix_attn(handle, layer: int, q, k, v, out, n_frames: int, use
            "ca2_spatial_prefix_attn")
 
 
+def ca2_tpe_add(handle, first_global_frame: int, offset: int, table, x, out, n_frames: int, stream=None) -> None:
+    _check(load_library().ca2_tpe_add(handle, int(first_global_frame), int(offset), _ptr(table), _ptr(x), _ptr(out),
+                                      int(n_frames), _stream(stream)),
+           "ca2_tpe_add")
+
+
 def ca2_tpe_indices(handle, first_global_frame: int, offset: int, n: int) -> List[int]:
     buf = (ctypes.c_int * max(1, n))()
     _check(load_library().ca2_tpe_indices(handle, int(first_global_frame), int(offset), int(n),
@@ -236,6 +243,7 @@ class KVCache:
                  tpe_len=0, device=None):
         import torch
         self.cfg = ca2_config(n_layers, batch, hw, heads, head_dim, chunk_len, p_max, p_spatial, tpe_len)
+        self.tpe_len = tpe_len if tpe_len > 0 else p_max + chunk_len   # rows of the TPE table
         tb, sb = ca2_cache_bytes(self.cfg)
         dev = device or torch.device("cuda", torch.cuda.current_device())
         self.tbuf = torch.empty(tb // 2, dtype=torch.bfloat16, device=dev)
@@ -291,3 +299,6 @@ class KVCache:
 
     def tpe(self, first_global_frame, offset, n):
         return ca2_tpe_indices(self.handle, first_global_frame, offset, n)
+
+    def tpe_add(self, first_global_frame, offset, table, x, out, n, stream=None):
+        ca2_tpe_add(self.handle, first_global_frame, offset, table, x, out, n, stream)

@@ -333,6 +333,28 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     return cuda_status(ca2::launch_spatial(m, p, static_cast<cudaStream_t>(stream)));
 }
 
+int ca2_tpe_add(const ca2_cache *c, long long first_global_frame, int offset, const void *table, const void *x,
+                void *out, int n, void *stream)
+{
+    if (!c || !table || !x || !out) return CA2_ERR_ARG;
+    if (first_global_frame < 0 || offset < 0) return CA2_ERR_ARG;
+    if (n < 1 || n > c->cfg.chunk_len) return CA2_ERR_SHAPE;
+    if (!aligned16(table) || !aligned16(x) || !aligned16(out)) return CA2_ERR_ALIGN;
+    const ca2_config &g = c->cfg;
+    const long long n_tpe = g.tpe_len;
+    ca2::TpeAddParams p;
+    p.x = static_cast<const uint4 *>(x);
+    p.out = static_cast<uint4 *>(out);
+    p.table = static_cast<const uint4 *>(table);
+    p.rows = (long long)g.batch * g.hw * n;
+    p.row_vec = g.heads * g.head_dim / 8;
+    p.n = n;
+    if (p.rows * p.row_vec >= (1ll << 31)) return CA2_ERR_SHAPE;   // the kernel indexes in 32 bits
+    for (int i = 0; i < ca2::kMaxChunk; ++i)
+        p.tpe_row[i] = i < n ? (int)(((long long)offset + first_global_frame + i) % n_tpe) : 0;
+    return cuda_status(ca2::launch_tpe_add(p, static_cast<cudaStream_t>(stream)));
+}
+
 int ca2_tpe_indices(const ca2_cache *c, long long first_global_frame, int offset, int n, int *out_host)
 {
     if (!c) return CA2_ERR_ARG;

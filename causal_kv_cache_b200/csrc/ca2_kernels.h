@@ -103,6 +103,19 @@ struct SpatialMaps {
 uint32_t spatial_smem_bytes(int D);
 cudaError_t launch_spatial(const SpatialMaps &maps, const SpatialParams &p, cudaStream_t stream);
 
+// ---- cyclic TPE added to a chunk ------------------------------------------------------------
+struct TpeAddParams {
+    const uint4 *x;         // token-major chunk [B][HW][n][C] (16-byte vectors)
+    uint4 *out;             // same layout; may equal x
+    const uint4 *table;     // [N_tpe][C]
+    long long rows;         // B * HW * n
+    int row_vec;            // 16-byte vectors per row of C = H*D elements
+    int n;                  // chunk frames
+    int tpe_row[kMaxChunk]; // table row of each chunk frame
+};
+
+cudaError_t launch_tpe_add(const TpeAddParams &p, cudaStream_t stream);
+
 // ---- bounded-wait self test ---------------------------------------------------------------
 cudaError_t launch_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
 int read_and_clear_status(int *status);

@@ -134,6 +134,21 @@ int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k,
 int ca2_spatial_prefix_attn(ca2_cache *cache, int layer, const void *q, const void *k,
                             const void *v, void *out, int n_frames, int use_prefix, void *stream);
 
+/* Cyclic temporal positional embedding added to a chunk (papernotes page, 关键设计 4,
+ * Cyclic-TPEs): frame c of the chunk (global frame first_global_frame + c) gets row
+ *   (offset + first_global_frame + c) mod N_tpe
+ * of `table` added to every token's C = H*D vector:
+ *   out[b][s][c][:] = round_bf16(x[b][s][c][:] + table[row(c)][:])
+ * The sum is taken in float32 and rounded once (nearest, ties to even).
+ * table: device, [N_tpe][H][D] bf16 (N_tpe = the cache's tpe_len), read only.
+ * x, out: device, token-major [B][HW][n][H][D] (the temporal branch's layout); out may be
+ * x itself (in place), otherwise they must not overlap.  1 <= n <= l.  All three 16-byte
+ * aligned.  Asynchronous on `stream`; the cache state is not touched.
+ * Errors: ARG (null pointer, negative frame or offset), SHAPE (n, or a chunk of 2^35 bytes or
+ * more), ALIGN, CUDA. */
+int ca2_tpe_add(const ca2_cache *cache, long long first_global_frame, int offset, const void *table,
+                const void *x, void *out, int n_frames, void *stream);
+
 /* Cyclic temporal positional-embedding indices (papernotes page, 关键设计 4, Cyclic-TPEs):
  * out_host[c] = (offset + first_global_frame + c) mod N_tpe for c < n.  Host-only.
  * first_global_frame >= 0, offset >= 0, n >= 0; out_host may be NULL only when n = 0. */

@@ -138,6 +138,13 @@ def test_call_validation_before_any_launch():
     with pytest.raises(ca2.Ca2Error) as e:
         ca2.ca2_cache_write(h, [al + 4], [al], [al], [al], 8, stream=0)
     assert e.value.status == -4
+    # TPE add checks: null pointers, negative frame/offset, frame count, alignment
+    for args, code in (((0, 0, None, al, al, 8), -1), ((0, 0, al, al, None, 8), -1), ((-1, 0, al, al, al, 8), -1),
+                       ((0, -3, al, al, al, 8), -1), ((0, 0, al, al, al, 0), -2), ((0, 0, al, al, al, 9), -2),
+                       ((0, 0, al + 8, al, al, 8), -4), ((0, 0, al, al, al + 2, 8), -4)):
+        with pytest.raises(ca2.Ca2Error) as e:
+            ca2.ca2_tpe_add(h, *args, stream=0)
+        assert e.value.status == code, args
     ca2.ca2_cache_destroy(h)
     # capacity: Pmax = 8 = l; a full chunk fits once, the next needs eviction first
     h2, _ = make(p_max=8)

@@ -8,6 +8,7 @@ import dataclasses
 import numpy as np
 import pytest
 
+import oracle
 from ca2_synth import WORKLOADS, Generator
 
 pytestmark = pytest.mark.gpu
@@ -195,6 +196,29 @@ def test_spatial_max_grows_in_late_blocks(head_dim):
     lp.write([kt], [vt], [bf16_bits(ks)], [vs])
     q, k, v = lp.gen.qkv(3)
     lp.spatial(0, q, k, v, use_prefix=1)
+
+
+@pytest.mark.parametrize("name,offset,g0", [("tiny", 0, 0), ("tiny", 3, 7), ("os_p41", 0, 41), ("os_p41", 17, 45)])
+def test_tpe_add_bit_exact(name, offset, g0):
+    """Chunk + cyclic TPE rows, out of place and in place, bit for bit against the oracle
+    (indices wrap past N_tpe for the larger first frames)."""
+    import torch
+    from causal_kv_cache_b200.ca2 import KVCache
+    from tests.gpu_util import to_bits, to_dev, token_major
+    wl = WORKLOADS[name]
+    g = Generator(wl, 11)
+    c = KVCache(1, wl.batch, wl.hw, wl.heads, wl.head_dim, wl.chunk_len, wl.p_max, wl.p_spatial)
+    C = wl.heads * wl.head_dim
+    table = g.frames(c.tpe_len)[0, :, 0].reshape(c.tpe_len, wl.heads, wl.head_dim)   # [N_tpe][H][D]
+    for n in (wl.chunk_len, 1):
+        x = token_major(g.frames(n))                                                  # [B][HW][n][H][D]
+        ref = oracle.tpe_add(x.reshape(wl.batch, wl.hw, n, C), table.reshape(-1, C), g0, offset)
+        xd, td = to_dev(x), to_dev(table)
+        out = torch.empty_like(xd)
+        c.tpe_add(g0, offset, td, xd, out, n)
+        assert np.array_equal(to_bits(out).reshape(ref.shape), ref)
+        c.tpe_add(g0, offset, td, xd, xd, n)                                          # in place
+        assert np.array_equal(to_bits(xd).reshape(ref.shape), ref)
 
 
 def test_multi_layer_write_bit_exact():
