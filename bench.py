@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--denoise", type=int, default=WORKLOAD["denoise_steps"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="step", choices=["step", "recompute"],
+                    help="step: the timed AR step (default); recompute: cached vs recompute-from-scratch "
+                         "attention per denoising step along the 80-frame run")
     return ap.parse_args()
 
 
@@ -519,10 +522,104 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+def run_recompute(args):
+    """Attention time per denoising step of one block along the 80-frame run: with the shared
+    cache (Ca2-VDM: the chunk's 8 frames attend to the queue) against recomputing every frame
+    of the window from scratch (OS-Ext style: each prefix frame again goes through spatial
+    self-attention and causal temporal attention over the frames before it).  The pages report
+    cumulative time linear in the AR step for the cached model and quadratic for recompute until
+    Pmax is reached ("Ca2-VDM" papernotes page, 实验结果, 关键发现 1; bohrium page, surprising
+    findings).  Attention only: projections and MLPs need the weights.  One JSON line."""
+    import torch
+    from causal_kv_cache_b200 import ca2
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, HW, H, D, l, PM, PS = (WORKLOAD[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max", "p_spatial"))
+    T = args.denoise
+    g = torch.Generator(device=dev)
+    g.manual_seed(77)
+    rnd = lambda *shape: (torch.randn(shape, generator=g, device=dev) * 0.7).to(torch.bfloat16)
+    steps = list(range(1, 11))                                   # AR steps of the 80-frame run
+    prefix = [min(8 * (k - 1) + 1, PM) for k in steps]           # queued frames before each step
+    qlens = sorted({0} | {q for P in prefix for q in [P] + list(range(1, P, 8))})
+    caches = {}
+    for q in qlens:                                              # one cache per queue length
+        c = ca2.KVCache(1, B, HW, H, D, l, PM, PS)
+        sizes = ([1] if q >= 1 else []) + [8] * ((q - 1) // 8 if q > 1 else 0)
+        for n in sizes:
+            kt, ks = rnd(B, HW, n, H, D), rnd(B, n, HW, H, D)
+            c.evict_for(n)
+            c.write([kt], [kt], [ks], [ks], n)
+        assert c.state()[1] == q
+        caches[q] = c
+    tq, tk, tv = (rnd(B, HW, l, H, D) for _ in range(3))
+    sq, sk, sv = (rnd(B, l, HW, H, D) for _ in range(3))
+    to, so = torch.empty_like(tq), torch.empty_like(sq)
+    tq1, tk1, tv1 = (rnd(B, HW, 1, H, D) for _ in range(3))
+    sq1, sk1, sv1 = (rnd(B, 1, HW, H, D) for _ in range(3))
+    to1, so1 = torch.empty_like(tq1), torch.empty_like(sq1)
+    cap = torch.cuda.Stream(device=dev)
+
+    def cached_pass(P, sp):
+        c = caches[P]
+        c.spatial_attn(0, sq, sk, sv, so, l, 1, sp)               # prefix-enhanced, P' cache frames
+        c.temporal(0, tq, tk, tv, to, l, sp)
+
+    def recompute_pass(P, sp):
+        # the window: frame 0 (no earlier frame), then groups of 8 with queues 1, 9, ..., then the chunk
+        caches[0].spatial_attn(0, sq1, sk1, sv1, so1, 1, 0, sp)
+        caches[0].temporal(0, tq1, tk1, tv1, to1, 1, sp)
+        for q in list(range(1, P, 8)) + [P]:
+            caches[q].spatial_attn(0, sq, sk, sv, so, l, 0, sp)
+            caches[q].temporal(0, tq, tk, tv, to, l, sp)
+
+    def time_graph(fn, P, reps=20):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            gr.capture_begin()
+            fn(P, int(cap.cuda_stream))
+            gr.capture_end()
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            gr.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / reps                    # us per pass
+
+    cached_us = [time_graph(cached_pass, P) for P in prefix]
+    recompute_us = [time_graph(recompute_pass, P) for P in prefix]
+    assert ca2.ca2_device_status() == 0
+    NL = WORKLOAD["n_layers"]
+    cum_c, cum_r, acc_c, acc_r = [], [], 0.0, 0.0
+    for c_us, r_us in zip(cached_us, recompute_us):
+        acc_c += c_us * T * NL / 1e3                              # ms of attention over the AR step
+        acc_r += r_us * T * NL / 1e3
+        cum_c.append(round(acc_c, 2))
+        cum_r.append(round(acc_r, 2))
+    out = {"mode": "recompute", "metric": "attention us per denoising step of one block",
+           "unit": "us", "ar_steps": steps, "prefix_frames": prefix,
+           "cached_us": [round(x, 2) for x in cached_us], "recompute_us": [round(x, 2) for x in recompute_us],
+           "cumulative_ms": {"cached": cum_c, "recompute": cum_r, "blocks": NL, "denoise_steps": T},
+           "ratio_last_step": round(recompute_us[-1] / cached_us[-1], 2),
+           "config": {"workload": WORKLOAD_NAME, "batch": B, "tokens_per_frame": HW, "heads": H,
+                      "head_dim": D, "chunk_len": l, "p_max": PM, "p_spatial": PS},
+           "data": "synthetic (seeded N(0,0.49) bf16); attention only (projections and MLPs need weights)"}
+    print(json.dumps(out))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "recompute":
+        run_recompute(args)
     else:
         run_ca2(args)
 

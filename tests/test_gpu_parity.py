@@ -221,6 +221,19 @@ def test_tpe_add_bit_exact(name, offset, g0):
         assert np.array_equal(to_bits(xd).reshape(ref.shape), ref)
 
 
+def test_long_queue_pmax81():
+    """A queue of up to 81 frames (six 16-slot ring groups): first frame + 11 AR steps of 8,
+    filling the ring and then evicting; every attention output and cache write checked."""
+    from tests.gpu_util import Loop
+    wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, hw=64, heads=2, head_dim=72, batch=1,
+             chunk_len=8, p_max=81, p_spatial=3)
+    lp = Loop(wl, seed=31)
+    lp.first_frame()
+    for _ in range(11):
+        lp.ar_step(wl.chunk_len, 1)
+    assert lp.rings[0].count == 81
+
+
 def test_multi_layer_write_bit_exact():
     """One cache-write launch for many layers (more than one launch's layer table)."""
     from tests.gpu_util import Loop
