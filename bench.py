@@ -52,9 +52,10 @@ def parse():
     ap.add_argument("--denoise", type=int, default=WORKLOAD["denoise_steps"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="step", choices=["step", "recompute"],
+    ap.add_argument("--mode", default="step", choices=["step", "recompute", "per-timestep"],
                     help="step: the timed AR step (default); recompute: cached vs recompute-from-scratch "
-                         "attention per denoising step along the 80-frame run")
+                         "attention per denoising step along the 80-frame run; per-timestep: one shared "
+                         "cache vs one cache per denoising step (memory and AR-step time)")
     return ap.parse_args()
 
 
@@ -614,12 +615,114 @@ def run_recompute(args):
     print(json.dumps(out))
 
 
+def run_per_timestep(args):
+    """One cache shared by all T denoising steps (Ca2-VDM: prefix frames at tEmb(0)) against one
+    cache per denoising step (a per-timestep KV cache, as when prefix K/V depend on the noise
+    level).  Same kernels.  Shared: each AR step is T passes reading the one cache, the
+    cache-writing pass and one write.  Per-timestep: T passes, pass t reading cache t, and T
+    writes, since each step's K/V are stored at their own noise level ("Ca2-VDM" papernotes page,
+    关键设计 2 and 实验结果, 关键发现 4).  Reports the cache bytes and the AR-step time of both."""
+    import torch
+    from causal_kv_cache_b200 import ca2
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, HW, H, D, l, PM, PS = (WORKLOAD[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max", "p_spatial"))
+    NL, T = args.layers, args.denoise
+    g = torch.Generator(device=dev)
+    g.manual_seed(99)
+    rnd = lambda *shape: (torch.randn(shape, generator=g, device=dev) * 0.7).to(torch.bfloat16)
+
+    def filled_cache():
+        c = ca2.KVCache(NL, B, HW, H, D, l, PM, PS)
+        kt, ks = [rnd(B, HW, 1, H, D)] * NL, [rnd(B, 1, HW, H, D)] * NL
+        c.evict_for(1)
+        c.write(kt, kt, ks, ks, 1)
+        kt8, ks8 = [rnd(B, HW, l, H, D)] * NL, [rnd(B, l, HW, H, D)] * NL
+        for _ in range(5):                                      # queue of 41 frames
+            c.evict_for(l)
+            c.write(kt8, kt8, ks8, ks8, l)
+        return c
+
+    shared = filled_cache()
+    per_t = [filled_cache() for _ in range(T)]
+    tq = [rnd(B, HW, l, H, D) for _ in range(NL)]
+    sq = [rnd(B, l, HW, H, D) for _ in range(NL)]
+    to, so = [torch.empty_like(x) for x in tq], [torch.empty_like(x) for x in sq]
+    kt8, ks8 = [rnd(B, HW, l, H, D) for _ in range(NL)], [rnd(B, l, HW, H, D) for _ in range(NL)]
+    cap = torch.cuda.Stream(device=dev)
+
+    def one_pass(c, use_prefix, sp):
+        for L in range(NL):
+            c.spatial_attn(L, sq[L], sq[L], sq[L], so[L], l, use_prefix, sp)
+            c.temporal(L, tq[L], tq[L], tq[L], to[L], l, sp)
+
+    def graph_of(fn):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            gr.capture_begin()
+            fn(int(cap.cuda_stream))
+            gr.capture_end()
+        return gr
+
+    g_shared = graph_of(lambda sp: one_pass(shared, 1, sp))
+    g_shared_self = graph_of(lambda sp: one_pass(shared, 0, sp))
+    g_per = [graph_of(lambda sp, c=c: one_pass(c, 1, sp)) for c in per_t]
+    stream = torch.cuda.current_stream()
+    sp = int(stream.cuda_stream)
+
+    def step_shared():
+        for _ in range(T):
+            g_shared.replay()
+        g_shared_self.replay()
+        shared.evict_for(l)                                     # the queue stays full: evict 8, write 8
+        shared.write(kt8, kt8, ks8, ks8, l, sp)
+
+    def step_per():
+        for t in range(T):
+            g_per[t].replay()
+        for c in per_t:                                         # each step's K/V into its own cache
+            c.evict_for(l)
+            c.write(kt8, kt8, ks8, ks8, l, sp)
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    ms_shared = timed(step_shared)
+    ms_per = timed(step_per)
+    assert ca2.ca2_device_status() == 0
+    assert shared.state()[1] == PM and all(c.state()[1] == PM for c in per_t)
+    tb, sbb = ca2.ca2_cache_bytes(shared.cfg)
+    bytes_one = tb + sbb
+    out = {"mode": "per-timestep", "metric": "AR-step time (ms) and cache bytes", "unit": "ms",
+           "shared": {"ms_per_ar_step": round(ms_shared, 3), "cache_bytes": bytes_one, "caches": 1},
+           "per_timestep": {"ms_per_ar_step": round(ms_per, 3), "cache_bytes": bytes_one * T, "caches": T},
+           "time_ratio": round(ms_per / ms_shared, 3), "memory_ratio": T,
+           "config": {"workload": WORKLOAD_NAME, "blocks": NL, "denoise_steps": T, "batch": B,
+                      "tokens_per_frame": HW, "heads": H, "head_dim": D, "chunk_len": l, "p_max": PM,
+                      "p_spatial": PS},
+           "data": "synthetic (seeded N(0,0.49) bf16)"}
+    print(json.dumps(out))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.mode == "recompute":
         run_recompute(args)
+    elif args.mode == "per-timestep":
+        run_per_timestep(args)
     else:
         run_ca2(args)
 
