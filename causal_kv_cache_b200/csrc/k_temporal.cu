@@ -33,10 +33,12 @@
 //     then O^T += V^T P^T.  Each lane owns the same two query columns in both
 //     accumulators, so the online-softmax rescale is lane-local; movmatrix turns P^T
 //     into the B operand and O^T back into rows for the stores.
-//   * Ring rows that hold no queued frame (slots not yet queued, and rows past Pmax that
-//     the copy did not write) are masked; their V rows are zeroed in shared memory before
-//     use, so stale bits (of the caller's buffer or of an earlier stage) never reach the
-//     accumulator.
+//   * Ring rows that hold no queued frame are masked, and their V rows are zero, so stale
+//     bits (of the caller's buffer or of an earlier stage) never reach the accumulator.
+//     The producer zeroes the V rows past Pmax, which the ring copy does not write, before
+//     it arms the stage (off the consumers' path), so the consumers write shared memory
+//     (and fence it against the next copy into the stage) only for slots inside Pmax that
+//     hold no queued frame, which happens only while the queue fills.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -231,6 +233,18 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                     const int s0 = box * kKeys;
                     const int ns = min(kKeys, p.Pmax - s0);
                     const uint32_t run = (uint32_t)(ns * D * 2);
+                    if (ns < kKeys) {
+                        // V rows ns..15 of every head := 0 (generic-proxy writes, ordered before
+                        // the stage's arrive and before any later copy into the stage)
+                        const uint32_t pad16 = (uint32_t)((kKeys - ns) * D * 2) / 16u;
+                        for (uint32_t i = (uint32_t)lane; i < (uint32_t)G * pad16; i += 32u) {
+                            const uint32_t w = i / pad16;
+                            const uint32_t a = dst + L.kv_box + w * (uint32_t)(kKeys * D * 2) + run + 16u * (i - w * pad16);
+                            asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(a), "r"(0u) : "memory");
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
                     if (lane == 0) mbar_expect_tx(full_bar(slot), 2u * (uint32_t)G * run);
                     __syncwarp();
                     if (lane < 2 * G) {
@@ -352,12 +366,12 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         const bool v = sl < p.Pmax && age < p.Pk;
                         vis[hr][0] = vis[hr][1] = v;
                     }
-                    // rows that hold no queued frame (stale slots, and rows past Pmax that the
-                    // copy did not write): zero their V rows
+                    // slots inside Pmax that hold no queued frame: zero their V rows (the
+                    // producer has zeroed the rows past Pmax)
                     const int sl = box * kKeys + (lane & 15);
                     int age = sl - p.head;
                     if (age < 0) age += p.Pmax;
-                    zero_v = !(sl < p.Pmax && age < p.Pk);
+                    zero_v = sl < p.Pmax && age >= p.Pk;
                 }
                 if (!warp_wait(full_bar(slot), (stage / kStages) & 1, 104, abort_flag)) { ok = false; break; }
                 const uint32_t kbase = sbase + (uint32_t)slot * L.stage_bytes + head_kv;
@@ -367,6 +381,9 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         const uint32_t r0 = vbase + (uint32_t)lane * row;
                         for (int o = 0; o < D * 2; o += 16)
                             asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(r0 + o), "r"(0u) : "memory");
+                        // these generic-proxy writes must be ordered before the next copy
+                        // into this stage
+                        fence_proxy_async_smem();
                     }
                     __syncwarp();
                 }
@@ -435,9 +452,6 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         mma16816(acc[t], a0, 0u, a2, 0u, pb0, pb1);
                     }
                 }
-                // generic-proxy writes (the zeroed rows) must be ordered before the next
-                // TMA write into this stage
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar(slot));
             }

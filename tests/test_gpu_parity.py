@@ -57,6 +57,23 @@ def test_first_frame_temporal_returns_v_exactly():
         assert np.array_equal(to_bits(out), tv)
 
 
+def test_poisoned_buffers_never_reach_outputs():
+    """A freshly allocated cache buffer holds anything.  With every element of both cache
+    buffers set to a NaN bit pattern before the first write, ring slots that hold no queued
+    frame, rows past Pmax of the last 16-slot group (Pmax = 41), and spatial-cache frames
+    not yet written must never reach an output: every output is finite and matches the
+    oracle while the queue fills."""
+    import torch
+    from tests.gpu_util import Loop
+    wl = _wl("os_p41", n_layers=1)
+    lp = Loop(wl, seed=21)
+    lp.cache.tbuf.view(torch.int16).fill_(0x7FC0)     # bf16 quiet NaN
+    lp.cache.sbuf.view(torch.int16).fill_(0x7FC0)
+    lp.first_frame()
+    for _ in range(3):
+        lp.ar_step(wl.chunk_len, 1)
+
+
 def test_os_p41_eighty_frames():
     """Open-Sora-shaped layer, Pmax = 41: first frame + 10 chunks of 8 (eviction from the
     7th write on) with a random cyclic TPE offset.  Temporal outputs in full at every call;
