@@ -30,7 +30,11 @@ inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 bloc
 }
 
 // ---- causal temporal attention ---------------------------------------------------------
-constexpr int kMaxTemporalGroup = 4;   // heads per work item = consumer warps per CTA
+// heads per work item = consumer warps per CTA.  Two heads and four stages make CTAs of
+// ~42 KB of shared memory at D = 72, five per SM: more independent consumer warps per SM
+// measured faster than deeper rings in fewer CTAs (each consumer handles its stages one
+// after another, so the number of consumers in flight sets the rate).
+constexpr int kMaxTemporalGroup = 2;
 constexpr int kMaxChunk = 8;           // queries per (token, head): the chunk length limit
 
 struct TemporalParams {

@@ -49,7 +49,7 @@ namespace ca2 {
 
 namespace {
 
-constexpr int kStages = 5;       // K+V stages in flight per CTA
+constexpr int kStages = 4;       // K+V stages in flight per CTA
 constexpr int kKeys = 16;        // key frames per stage
 constexpr int kQ = 8;            // queries per (token, head): the mma N extent
 
