@@ -32,7 +32,10 @@
 //     products use mma.sync on registers: S^T = K Q^T (keys on M, the 8 queries on N),
 //     then O^T += V^T P^T.  Each lane owns the same two query columns in both
 //     accumulators, so the online-softmax rescale is lane-local; movmatrix turns P^T
-//     into the B operand and O^T back into rows for the stores.
+//     into the B operand and O^T back into rows for the stores.  The reference max of the
+//     exponentials moves only when a score exceeds it by more than 2^8 (one warp vote per
+//     stage; the max reduction and the rescale run only then), which leaves each softmax
+//     row unchanged after normalisation.
 //   * Ring rows that hold no queued frame are masked, and their V rows are zero, so stale
 //     bits (of the caller's buffer or of an earlier stage) never reach the accumulator.
 //     The producer zeroes the V rows past Pmax, which the ring copy does not write, before
@@ -52,6 +55,7 @@ namespace {
 constexpr int kStages = 4;       // K+V stages in flight per CTA
 constexpr int kKeys = 16;        // key frames per stage
 constexpr int kQ = 8;            // queries per (token, head): the mma N extent
+constexpr float kLazy = 8.0f;    // log2 units
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
@@ -410,30 +414,35 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                 sc[3] = vis[1][1] ? c[3] * p.scale_log2 : neg_inf;
                 float mx0 = fmaxf(sc[0], sc[2]);
                 float mx1 = fmaxf(sc[1], sc[3]);
+                // the reference max moves only when a score exceeds it by more than 2^8 (always
+                // on stage 0, which holds chunk frame 0, visible to every query)
+                if (__any_sync(0xffffffffu, mx0 > m_run[0] + kLazy || mx1 > m_run[1] + kLazy)) {
 #pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    }
+                    const float mn0 = fmaxf(m_run[0], mx0);
+                    const float mn1 = fmaxf(m_run[1], mx1);
+                    const float al0 = ex2(m_run[0] - mn0);
+                    const float al1 = ex2(m_run[1] - mn1);
+                    m_run[0] = mn0;
+                    m_run[1] = mn1;
+                    l_part[0] *= al0;
+                    l_part[1] *= al1;
+#pragma unroll
+                    for (int t = 0; t < DT; ++t) {
+                        acc[t][0] *= al0;
+                        acc[t][1] *= al1;
+                        acc[t][2] *= al0;
+                        acc[t][3] *= al1;
+                    }
                 }
-                // stage 0 holds chunk frame 0, visible to every query: m_run is finite after it
-                const float mn0 = fmaxf(m_run[0], mx0);
-                const float mn1 = fmaxf(m_run[1], mx1);
-                const float al0 = ex2(m_run[0] - mn0);
-                const float al1 = ex2(m_run[1] - mn1);
-                m_run[0] = mn0;
-                m_run[1] = mn1;
                 // probabilities rounded to bf16; the normaliser sums the rounded values
-                const uint32_t x0 = pack_bf16x2(ex2(sc[0] - mn0), ex2(sc[1] - mn1));
-                const uint32_t x1 = pack_bf16x2(ex2(sc[2] - mn0), ex2(sc[3] - mn1));
-                l_part[0] = l_part[0] * al0 + (bf16_lo(x0) + bf16_lo(x1));
-                l_part[1] = l_part[1] * al1 + (bf16_hi(x0) + bf16_hi(x1));
-#pragma unroll
-                for (int t = 0; t < DT; ++t) {
-                    acc[t][0] *= al0;
-                    acc[t][1] *= al1;
-                    acc[t][2] *= al0;
-                    acc[t][3] *= al1;
-                }
+                const uint32_t x0 = pack_bf16x2(ex2(sc[0] - m_run[0]), ex2(sc[1] - m_run[1]));
+                const uint32_t x1 = pack_bf16x2(ex2(sc[2] - m_run[0]), ex2(sc[3] - m_run[1]));
+                l_part[0] += bf16_lo(x0) + bf16_lo(x1);
+                l_part[1] += bf16_hi(x0) + bf16_hi(x1);
                 const uint32_t pb0 = movm_t(x0);
                 const uint32_t pb1 = movm_t(x1);
                 // O^T += V^T P^T, 16 head dims per m-tile
