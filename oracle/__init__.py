@@ -24,6 +24,12 @@ What it holds (all plain definitions, fp64 for floating point, integers exact):
   rounding to bf16 (nearest, ties to even), the precision the kernel computes in.
 * ``cache_bytes``    -- bytes of the shared KV cache (K and V, 2-byte elements,
   Pmax temporal frames plus P' spatial frames per layer).
+* ``kv_projection``  -- the K and V a layer stores in the cache-writing stage: the clean
+  chunk's hidden states times the layer's K and V projection weights, plus a bias
+  (papernotes page, 整体框架: one forward pass over the denoised chunk computes the new KV
+  cache; 关键设计 1: attention over Q, K, V).  The weight is one [2C][C] matrix, K rows
+  first (the nn.Linear layout).  Exact in fp64; ``kv_projection_bound`` gives the
+  magnitude sum an fp32 accumulation error is measured against.
 
 Parity status: every function is pinned by tests in ``tests/test_oracle_pins.py``
 (brute-force full-sequence attention, library SDPA special cases, closed forms, the
@@ -204,6 +210,41 @@ def tpe_add(x: np.ndarray, table: np.ndarray, first_global_frame: int, offset: i
     xf = (x.astype(np.uint32) << 16).view(np.float32)
     tf = (table.astype(np.uint32) << 16).view(np.float32)[idx]          # [n][C]
     return bf16_round_bits(xf + tf[None, None, :, :])
+
+
+def kv_projection(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray] = None):
+    """K and V of one layer from its input rows: x [rows][C], w [2C][C], b [2C] or None,
+    all bf16 bits.  Returns (K, V), each [rows][C] float64: Y = x w^T + b, K = Y[:, :C],
+    V = Y[:, C:] (papernotes page, 整体框架 and 关键设计 1).  Every product of two bf16
+    values is exact in fp64 and the sum carries fp64 rounding only (2^-53 relative per
+    term), far below the fp32 accumulation error the kernel is compared with.
+    """
+    xf = _bits_to_f64(x)
+    wf = _bits_to_f64(w)
+    C = xf.shape[1]
+    if wf.shape != (2 * C, C):
+        raise ValueError("w must be [2C][C] with the rows' C")
+    y = xf @ wf.T
+    if b is not None:
+        bf = _bits_to_f64(b)
+        if bf.shape != (2 * C,):
+            raise ValueError("b must be [2C]")
+        y = y + bf[None, :]
+    return y[:, :C], y[:, C:]
+
+
+def kv_projection_bound(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray] = None) -> np.ndarray:
+    """sum_i |x_i w_oi| + |b_o| for every output element, [rows][2C] float64: the scale of
+    the rounding error of any summation order of the projection."""
+    y = np.abs(_bits_to_f64(x)) @ np.abs(_bits_to_f64(w)).T
+    if b is not None:
+        y = y + np.abs(_bits_to_f64(b))[None, :]
+    return y
+
+
+def _bits_to_f64(a: np.ndarray) -> np.ndarray:
+    a = _u16(a)
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def cache_bytes(n_layers: int, batch: int, hw: int, heads: int, head_dim: int,

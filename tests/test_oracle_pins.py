@@ -198,3 +198,54 @@ def test_tpe_add_rounds_ties_to_even():
     x = _bits([1.0, 1.0078125, 1.0]).reshape(1, 1, 1, 3)
     out = oracle.tpe_add(x, table, 0, 0)
     assert out.reshape(-1).tolist() == [0x3F80, 0x3F82, 0x3F81]   # 1.0, 1.015625, 1.0078125
+
+
+def _bf16_bits(vals):
+    """Small exactly representable values -> bf16 bits."""
+    f = np.asarray(vals, dtype=np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_kv_projection_matches_brute_force_loops():
+    """Y[r][o] = sum_i x[r][i] w[o][i] + b[o] written out as loops on a tiny case (integer
+    values: exact in any order); K is output channels 0..C-1, V channels C..2C-1.  A
+    transposed weight, a swapped K/V half or a dropped bias fails it."""
+    rng = np.random.default_rng(5)
+    rows, C = 3, 4
+    x = rng.integers(-4, 5, size=(rows, C))
+    w = rng.integers(-3, 4, size=(2 * C, C))
+    b = rng.integers(-8, 9, size=(2 * C,))
+    k, v = oracle.kv_projection(_bf16_bits(x), _bf16_bits(w), _bf16_bits(b))
+    for r in range(rows):
+        for o in range(2 * C):
+            acc = float(b[o])
+            for i in range(C):
+                acc += float(x[r][i]) * float(w[o][i])
+            got = k[r][o] if o < C else v[r][o - C]
+            assert got == acc, (r, o, got, acc)
+
+
+def test_kv_projection_identity_and_bias_only():
+    """W = [I; 2I] with no bias returns K = x and V = 2x exactly; W = 0 returns the bias."""
+    rng = np.random.default_rng(6)
+    C = 8
+    x = _bf16_bits(rng.integers(-64, 65, size=(5, C)) / 16.0)
+    eye = np.eye(C, dtype=np.float32)
+    k, v = oracle.kv_projection(x, _bf16_bits(np.concatenate([eye, 2 * eye])))
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(k, xf) and np.array_equal(v, 2 * xf)
+    b = rng.integers(-8, 9, size=(2 * C,)).astype(np.float32)
+    k, v = oracle.kv_projection(x, _bf16_bits(np.zeros((2 * C, C))), _bf16_bits(b))
+    assert np.array_equal(k, np.broadcast_to(b[:C], (5, C))) and np.array_equal(v, np.broadcast_to(b[C:], (5, C)))
+
+
+def test_kv_projection_bound_is_the_magnitude_sum():
+    """The bound is sum_i |x_i w_oi| + |b_o|: on sign-mixed integers it exceeds |Y| and
+    equals it when every term is positive."""
+    x = _bf16_bits([[1, -2, 3]])
+    w = _bf16_bits([[1, 1, 1], [2, 0, -1], [-1, -1, -1], [0, 1, 0], [1, 2, 3], [3, 2, 1]])
+    b = _bf16_bits([1, -1, 0, 2, 0, 0])
+    bound = oracle.kv_projection_bound(x, w, b)
+    assert bound.tolist() == [[7.0, 6.0, 6.0, 4.0, 14.0, 10.0]]
+    k, v = oracle.kv_projection(x, w, b)
+    assert np.all(np.abs(np.concatenate([k, v], axis=1)) <= bound)
