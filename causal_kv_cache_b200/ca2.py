@@ -18,7 +18,8 @@ from typing import List, Optional, Sequence, Tuple
 __all__ = [
     "Ca2Error", "ca2_config", "load_library", "LIBRARY_PATH",
     "ca2_cache_bytes", "ca2_cache_init", "ca2_cache_destroy", "ca2_cache_evict",
-    "ca2_cache_write", "ca2_temporal_attn", "ca2_spatial_prefix_attn", "ca2_tpe_indices", "ca2_tpe_add",
+    "ca2_cache_write", "ca2_kv_proj_write", "ca2_cache_commit", "ca2_temporal_attn", "ca2_spatial_prefix_attn",
+    "ca2_tpe_indices", "ca2_tpe_add",
     "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string",
     "ca2_last_error_string",
     "KVCache", "STATUS",
@@ -76,6 +77,8 @@ def load_library(path: Optional[str] = None):
         "ca2_cache_destroy": ([vp], i),
         "ca2_cache_evict": ([vp, i], i),
         "ca2_cache_write": ([vp, pp, pp, pp, pp, i, vp], i),
+        "ca2_kv_proj_write": ([vp, i, vp, vp, vp, vp, vp, vp, i, vp], i),
+        "ca2_cache_commit": ([vp, i], i),
         "ca2_temporal_attn": ([vp, i, vp, vp, vp, vp, i, vp], i),
         "ca2_spatial_prefix_attn": ([vp, i, vp, vp, vp, vp, i, i, vp], i),
         "ca2_tpe_indices": ([vp, ll, i, i, ctypes.POINTER(ctypes.c_int)], i),
@@ -176,6 +179,16 @@ def ca2_cache_write(handle, k_t, v_t, k_s, v_s, n_frames: int, stream=None) -> N
     _check(load_library().ca2_cache_write(handle, _ptr_array(k_t), _ptr_array(v_t), _ptr_array(k_s),
                                           _ptr_array(v_s), int(n_frames), _stream(stream)),
            "ca2_cache_write")
+
+
+def ca2_kv_proj_write(handle, layer: int, x_t, w_t, b_t, x_s, w_s, b_s, n_frames: int, stream=None) -> None:
+    _check(load_library().ca2_kv_proj_write(handle, int(layer), _ptr(x_t), _ptr(w_t), _ptr(b_t), _ptr(x_s),
+                                            _ptr(w_s), _ptr(b_s), int(n_frames), _stream(stream)),
+           "ca2_kv_proj_write")
+
+
+def ca2_cache_commit(handle, n_frames: int) -> None:
+    _check(load_library().ca2_cache_commit(handle, int(n_frames)), "ca2_cache_commit")
 
 
 def ca2_temporal_attn(handle, layer: int, q, k, v, out, n_frames: int, stream=None) -> None:
@@ -290,6 +303,12 @@ class KVCache:
 
     def write(self, k_t, v_t, k_s, v_s, n, stream=None):
         ca2_cache_write(self.handle, k_t, v_t, k_s, v_s, n, stream)
+
+    def kv_proj_write(self, layer, x_t, w_t, b_t, x_s, w_s, b_s, n, stream=None):
+        ca2_kv_proj_write(self.handle, layer, x_t, w_t, b_t, x_s, w_s, b_s, n, stream)
+
+    def commit(self, n):
+        ca2_cache_commit(self.handle, n)
 
     def temporal(self, layer, q, k, v, out, n, stream=None):
         ca2_temporal_attn(self.handle, layer, q, k, v, out, n, stream)

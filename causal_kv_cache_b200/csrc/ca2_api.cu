@@ -122,6 +122,23 @@ bool encode_5d(CUtensorMap *m, const void *base, int D, int frames, int H, int H
     return r == CUDA_SUCCESS;
 }
 
+// 3-D view (channel, row, plane) of a bf16 matrix stack with the given row and plane
+// strides (elements); box 64 channels x box_rows x 1, 128-byte swizzle (GEMM operand tiles).
+bool encode_rows_3d(CUtensorMap *m, const void *base, long long cols, long long rows, long long planes,
+                    long long row_stride, long long plane_stride, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)planes};
+    cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)plane_stride * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 uint8_t *layer_ring(const ca2_cache *c, int layer, int kv)
 {
     return c->tbuf + ((size_t)layer * 2 + (size_t)kv) * (size_t)c->cfg.p_max * c->plane_bytes;
@@ -331,6 +348,77 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     p.q_pairs = (g.hw + 255) / 256;
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
     return cuda_status(ca2::launch_spatial(m, p, static_cast<cudaStream_t>(stream)));
+}
+
+int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t, const void *b_t, const void *x_s,
+                      const void *w_s, const void *b_s, int n, void *stream)
+{
+    if (!c || !x_t || !w_t) return CA2_ERR_ARG;
+    const ca2_config &g = c->cfg;
+    if (layer < 0 || layer >= g.n_layers) return CA2_ERR_ARG;
+    if (n < 1 || n > g.chunk_len) return CA2_ERR_SHAPE;
+    if (c->count + n > g.p_max) return CA2_ERR_CAPACITY;
+    const int n_sp = n < g.p_spatial ? n : g.p_spatial;
+    if (n_sp > 0 && (!x_s || !w_s)) return CA2_ERR_ARG;
+    const void *ptrs[6] = {x_t, w_t, b_t, n_sp > 0 ? x_s : nullptr, n_sp > 0 ? w_s : nullptr, n_sp > 0 ? b_s : nullptr};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return CA2_ERR_ALIGN;
+    const long long C = (long long)g.heads * g.head_dim;
+    const long long rows_t = (long long)g.batch * g.hw * n;
+    if (rows_t >= (1ll << 31) || C * 2 >= (1ll << 31)) return CA2_ERR_SHAPE;
+
+    ca2::KvProjParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.ring_k = reinterpret_cast<__nv_bfloat16 *>(layer_ring(c, layer, 0));
+    p.ring_v = reinterpret_cast<__nv_bfloat16 *>(layer_ring(c, layer, 1));
+    p.sp_k = n_sp > 0 ? reinterpret_cast<__nv_bfloat16 *>(layer_spatial(c, layer, 0)) : nullptr;
+    p.sp_v = n_sp > 0 ? reinterpret_cast<__nv_bfloat16 *>(layer_spatial(c, layer, 1)) : nullptr;
+    p.bias_t = static_cast<const __nv_bfloat16 *>(b_t);
+    p.bias_s = n_sp > 0 ? static_cast<const __nv_bfloat16 *>(b_s) : nullptr;
+    p.B = g.batch;
+    p.HW = g.hw;
+    p.H = g.heads;
+    p.D = g.head_dim;
+    p.C = (int)C;
+    p.n = n;
+    p.p_max = g.p_max;
+    p.slot0 = (c->head + c->count) % g.p_max;
+    p.n_sp = n_sp;
+    p.rows_t = (int)rows_t;
+    p.tiles_n = (int)((2 * C + 255) / 256);
+    p.tiles_t = (int)((rows_t + 127) / 128) * p.tiles_n;
+    p.tiles_s_frame = (g.hw + 127) / 128;
+    p.k_steps = (int)((C + 63) / 64);
+    const long long tiles_s = (long long)g.batch * n_sp * p.tiles_s_frame * p.tiles_n;
+    if (p.tiles_t + tiles_s >= (1ll << 31)) return CA2_ERR_SHAPE;
+
+    // x_t: [B*HW*n][C]; x_s: (C, HW, B*n frames); W: [2C][C] (output channel rows)
+    ca2::KvProjMaps m;
+    std::memset(&m, 0, sizeof(m));
+    bool ok = encode_rows_3d(&m.xt, x_t, C, rows_t, 1, C, rows_t * C, 128) &&
+              encode_rows_3d(&m.wt, w_t, C, 2 * C, 1, C, 2 * C * C, 256);
+    if (ok && n_sp > 0)
+        ok = encode_rows_3d(&m.xs, x_s, C, g.hw, (long long)g.batch * n, C, (long long)g.hw * C, 128) &&
+             encode_rows_3d(&m.ws, w_s, C, 2 * C, 1, C, 2 * C * C, 256);
+    else
+        m.xs = m.xt, m.ws = m.wt;    // no spatial tile reads them
+    if (!ok) {
+        g_last_cuda_error = "tensor-map encoding failed";
+        return CA2_ERR_CUDA;
+    }
+    return cuda_status(ca2::launch_kv_proj(m, p, (int)(p.tiles_t + tiles_s), static_cast<cudaStream_t>(stream)));
+}
+
+int ca2_cache_commit(ca2_cache *c, int n)
+{
+    if (!c) return CA2_ERR_ARG;
+    const ca2_config &g = c->cfg;
+    if (n < 1 || n > g.chunk_len) return CA2_ERR_SHAPE;
+    if (c->count + n > g.p_max) return CA2_ERR_CAPACITY;
+    c->count += n;
+    c->sp_count = n < g.p_spatial ? n : g.p_spatial;
+    c->frames_written += n;
+    return CA2_OK;
 }
 
 int ca2_tpe_add(const ca2_cache *c, long long first_global_frame, int offset, const void *table, const void *x,

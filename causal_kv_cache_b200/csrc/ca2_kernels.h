@@ -120,6 +120,33 @@ struct TpeAddParams {
 
 cudaError_t launch_tpe_add(const TpeAddParams &p, cudaStream_t stream);
 
+// ---- K/V projection of the cache-writing stage, stored straight into the caches ----------
+// Output tiles of 128 rows x 256 channels over [K | V] (2C channels); temporal tiles first,
+// then spatial tiles.  Rows: temporal (b, s, f) of the token-major chunk input; spatial
+// (s) of one of the chunk's last n_sp frames.
+struct KvProjParams {
+    __nv_bfloat16 *ring_k, *ring_v;       // this layer's K and V rings [B][HW][H][Pmax][D]
+    __nv_bfloat16 *sp_k, *sp_v;           // this layer's spatial cache [P'][B][HW][H][D]
+    const __nv_bfloat16 *bias_t, *bias_s; // [2C] or null
+    int B, HW, H, D, C, n;
+    int p_max, slot0;       // ring slot of chunk frame 0
+    int n_sp;               // chunk frames stored in the spatial cache (the last n_sp)
+    int rows_t;             // B * HW * n
+    int tiles_n;            // ceil(2C / 256)
+    int tiles_t;            // temporal tiles: ceil(rows_t / 128) * tiles_n
+    int tiles_s_frame;      // spatial row tiles per frame: ceil(HW / 128)
+    int k_steps;            // ceil(C / 64)
+};
+
+// A tiles: boxes of 64 channels x 128 rows (x 1 frame); W tiles: 64 channels x 256 rows;
+// all with 128-byte rows and the 128-byte swizzle.  xt, wt: 3-D views with one plane;
+// xs: (channel, token, frame) of the frame-major chunk input.
+struct KvProjMaps {
+    CUtensorMap xt, wt, xs, ws;
+};
+
+cudaError_t launch_kv_proj(const KvProjMaps &maps, const KvProjParams &p, int grid, cudaStream_t stream);
+
 // ---- bounded-wait self test ---------------------------------------------------------------
 cudaError_t launch_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
 int read_and_clear_status(int *status);

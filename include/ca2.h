@@ -109,6 +109,29 @@ int ca2_cache_evict(ca2_cache *cache, int n_frames);
 int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const *v_t,
                     const void *const *k_s, const void *const *v_s, int n_frames, void *stream);
 
+/* Cache-writing stage fused into the K/V projection of one layer (papernotes page, 整体框架:
+ * the cache-writing stage is one forward pass over the denoised chunk that computes and
+ * stores the new KV cache; 关键设计 4 and 5: the temporal queue and the spatial cache).
+ *   temporal: [K | V] = x_t w_t^T + b_t for every row (b, s, f) of x_t; K and V of chunk
+ *             frame f go to ring slot (head + count + f) mod Pmax of layer `layer`;
+ *   spatial : [K | V] = x_s w_s^T + b_s for the chunk's last n_sp = min(P', n) frames of
+ *             x_s; frame f goes to spatial-cache frame f - (n - n_sp).
+ * x_t: token-major [B][HW][n][C] (C = H*D); x_s: frame-major [B][n][HW][C]; w_t, w_s:
+ * [2C][C] row-major, row o = output channel o (K channels 0..C-1 as (head, dim), then V);
+ * b_t, b_s: [2C] or NULL for no bias.  All bf16, device memory, 16-byte aligned.  fp32
+ * accumulation on the tensor cores, then the bias, then one rounding to bf16 (nearest,
+ * ties to even).  x_s, w_s, b_s are not read when n_sp = 0 (may be NULL).
+ * The queue does not advance: after this call for every layer, call ca2_cache_commit(n)
+ * (evict first, as for ca2_cache_write).  1 <= n <= chunk_len and count + n <= Pmax, else
+ * CA2_ERR_SHAPE / CA2_ERR_CAPACITY.  Asynchronous on `stream`. */
+int ca2_kv_proj_write(ca2_cache *cache, int layer, const void *x_t, const void *w_t, const void *b_t,
+                      const void *x_s, const void *w_s, const void *b_s, int n_frames, void *stream);
+
+/* Advance the queue after ca2_kv_proj_write of every layer: count += n, the spatial cache
+ * now holds min(P', n) frames, frames_written += n.  Host-only.  Same limits as
+ * ca2_kv_proj_write. */
+int ca2_cache_commit(ca2_cache *cache, int n_frames);
+
 /* Causal temporal attention of one layer (papernotes page, 关键设计 1, equation
  * CausalAttn; bohrium arXiv 2411.16375 page, formula with M_ij = -inf for i < j).
  * For every (b, s, h) and chunk frame c:

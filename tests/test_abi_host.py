@@ -172,3 +172,50 @@ def test_status_strings():
     for code in range(-6, 1):
         assert ca2.ca2_status_string(code) != "unknown status"
     assert ca2.ca2_status_string(-99) == "unknown status"
+
+
+def test_kv_proj_write_validation_and_commit():
+    """The fused projection write rejects bad arguments before any device work, and
+    ca2_cache_commit advances the queue exactly as a cache write of n frames does."""
+    h, c = make()
+    X, W, B = FAKE_T + 0x100000, FAKE_T + 0x200000, FAKE_T + 0x300000
+    bad = [
+        (dict(x_t=None), -1), (dict(w_t=None), -1), (dict(layer=1), -1), (dict(layer=-1), -1),
+        (dict(n=0), -2), (dict(n=9), -2), (dict(x_t=X + 8), -4), (dict(w_t=W + 2), -4),
+        (dict(b_t=B + 4), -4), (dict(x_s=None), -1), (dict(w_s=None), -1), (dict(x_s=X + 8), -4),
+    ]
+    for kw, status in bad:
+        a = dict(layer=0, x_t=X, w_t=W, b_t=B, x_s=X, w_s=W, b_s=None, n=8)
+        a.update(kw)
+        with pytest.raises(ca2.Ca2Error) as e:
+            ca2.ca2_kv_proj_write(h, a["layer"], a["x_t"], a["w_t"], a["b_t"], a["x_s"], a["w_s"], a["b_s"], a["n"])
+        assert e.value.status == status, (kw, e.value.status)
+    # commit: count += n, the spatial cache holds min(P', n) frames
+    ca2.ca2_cache_commit(h, 1)
+    assert ca2.ca2_cache_state(h) == (0, 1, 1, 1)
+    ca2.ca2_cache_commit(h, 8)
+    assert ca2.ca2_cache_state(h) == (0, 9, 3, 9)
+    for n, status in ((0, -2), (9, -2)):
+        with pytest.raises(ca2.Ca2Error) as e:
+            ca2.ca2_cache_commit(h, n)
+        assert e.value.status == status
+    ca2.ca2_cache_destroy(h)
+    # a write or commit past Pmax needs an eviction first
+    h, c = make(p_max=8)
+    ca2.ca2_cache_commit(h, 8)
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_kv_proj_write(h, 0, X, W, None, X, W, None, 1)
+    assert e.value.status == -3
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_cache_commit(h, 1)
+    assert e.value.status == -3
+    ca2.ca2_cache_evict(h, 1)
+    ca2.ca2_cache_commit(h, 1)
+    assert ca2.ca2_cache_state(h) == (1, 8, 1, 9)
+    ca2.ca2_cache_destroy(h)
+    # P' = 0: the spatial operands are not needed
+    h, c = make(p_spatial=0)
+    with pytest.raises(ca2.Ca2Error) as e:
+        ca2.ca2_kv_proj_write(h, 0, X + 8, W, None, None, None, None, 8)
+    assert e.value.status == -4
+    ca2.ca2_cache_destroy(h)

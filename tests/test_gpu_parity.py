@@ -294,3 +294,93 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert ca2.ca2_device_status() == 0
     x = torch.ones(4, device="cuda")
     assert float(x.sum()) == 4.0
+
+
+def _bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits), for normal x."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return np.exp2(e - 7)
+
+
+def _check_projection(got_bits, exact, bound, C, what):
+    """|got - exact| <= half a bf16 ulp (the one rounding) + the fp32 accumulation bound
+    C * 2^-23 * sum|x w| (twice the textbook gamma_C of recursive summation)."""
+    got = (got_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.isfinite(got).all(), "%s: non-finite value" % what
+    tol = 0.5 * _bf16_ulp(np.maximum(np.abs(exact), np.abs(got))) + C * 2.0 ** -23 * bound
+    err = np.abs(got - exact)
+    assert (err <= tol).all(), "%s: max excess %g" % (what, float((err - tol).max()))
+
+
+@pytest.mark.parametrize("shape,bias", [
+    (dict(n_layers=2, batch=1, hw=256, heads=16, head_dim=72, chunk_len=8, p_max=41, p_spatial=3), True),
+    (dict(n_layers=2, batch=2, hw=200, heads=3, head_dim=16, chunk_len=5, p_max=13, p_spatial=2), False),
+    (dict(n_layers=2, batch=1, hw=130, heads=4, head_dim=128, chunk_len=3, p_max=7, p_spatial=3, n=2), True),
+])
+def test_kv_proj_write_matches_oracle(shape, bias):
+    """The cache-writing stage's K/V projection stored straight into the caches: every
+    written element against the exact projection, every other ring slot, spatial frame and
+    layer untouched (still the poison), with the write wrapping past the ring's end."""
+    import torch
+    from causal_kv_cache_b200.ca2 import KVCache
+    s = dict(shape)
+    NL, B, HW, H, D, l, PM, PS = (s[k] for k in ("n_layers", "batch", "hw", "heads", "head_dim", "chunk_len",
+                                                "p_max", "p_spatial"))
+    n = s.get("n", l)                       # a short chunk: fewer frames than P' reach the spatial cache
+    C = H * D
+    rng = np.random.default_rng(31)
+    bits = lambda a: (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    n_sp = min(PS, n)
+    x_t = bits(rng.standard_normal((B, HW, n, C)))
+    x_s = bits(rng.standard_normal((B, n, HW, C)))
+    w_t = bits(rng.standard_normal((2 * C, C)) / np.sqrt(C))
+    w_s = bits(rng.standard_normal((2 * C, C)) / np.sqrt(C))
+    b_t = bits(rng.standard_normal(2 * C)) if bias else None
+    b_s = bits(rng.standard_normal(2 * C)) if bias else None
+    dev = lambda a: None if a is None else torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    cache = KVCache(NL, B, HW, H, D, l, PM, PS)
+    cache.tbuf.view(torch.int16).fill_(0x7FC0)
+    cache.sbuf.view(torch.int16).fill_(0x7FC0)
+    # move the ring head so that the chunk's slots wrap past the end of the ring
+    def advance(k):
+        while k > 0:
+            cache.commit(min(l, k))
+            k -= min(l, k)
+    advance(n)
+    cache.evict(n)
+    advance(max(1, PM - n - 1))
+    head, count = cache.state()[0], cache.state()[1]
+    if count + n > PM:
+        cache.evict(count + n - PM)
+    head, count = cache.state()[0], cache.state()[1]
+    slot0 = (head + count) % PM
+    cache.kv_proj_write(1, dev(x_t), dev(w_t), dev(b_t), dev(x_s), dev(w_s), dev(b_s), n)
+    torch.cuda.synchronize()
+    from causal_kv_cache_b200 import ca2
+    assert ca2.ca2_device_status() == 0
+    ring = [cache.ring(1, kv).view(torch.int16).cpu().numpy().view(np.uint16) for kv in (0, 1)]
+    spat = [cache.spatial(1, kv).view(torch.int16).cpu().numpy().view(np.uint16) for kv in (0, 1)]
+    # temporal: rows (b, s, f)
+    k, v = oracle.kv_projection(x_t.reshape(-1, C), w_t, b_t)
+    bound = oracle.kv_projection_bound(x_t.reshape(-1, C), w_t, b_t)
+    slots = [(slot0 + f) % PM for f in range(n)]
+    for kv, exact, bnd in ((0, k, bound[:, :C]), (1, v, bound[:, C:])):
+        got = ring[kv][:, :, :, slots, :]                       # [B][HW][H][n][D]
+        got = got.transpose(0, 1, 3, 2, 4).reshape(-1, C)       # rows (b, s, f), channels (h, d)
+        _check_projection(got, exact, bnd, C, "temporal %s" % "KV"[kv])
+        rest = np.delete(ring[kv], slots, axis=3)
+        assert (rest == 0x7FC0).all(), "temporal: a slot outside the chunk's was written"
+    # spatial: the chunk's last n_sp frames, rows (b, s) per frame
+    xs_last = x_s[:, n - n_sp:]                                 # [B][n_sp][HW][C]
+    k, v = oracle.kv_projection(xs_last.reshape(-1, C), w_s, b_s)
+    bound = oracle.kv_projection_bound(xs_last.reshape(-1, C), w_s, b_s)
+    for kv, exact, bnd in ((0, k, bound[:, :C]), (1, v, bound[:, C:])):
+        got = spat[kv][:n_sp].transpose(1, 0, 2, 3, 4).reshape(-1, C)   # [B][n_sp][HW] rows
+        _check_projection(got, exact, bnd, C, "spatial %s" % "KV"[kv])
+        assert (spat[kv][n_sp:] == 0x7FC0).all(), "spatial: a frame past n_sp was written"
+    # layer 0 untouched
+    for kv in (0, 1):
+        assert (cache.ring(0, kv).view(torch.int16) == 0x7FC0).all().item()
+        assert (cache.spatial(0, kv).view(torch.int16) == 0x7FC0).all().item()
+    cache.commit(n)
+    assert cache.state()[1] == count + n and cache.state()[2] == n_sp
