@@ -385,7 +385,7 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     p.slot0 = (c->head + c->count) % g.p_max;
     p.n_sp = n_sp;
     p.rows_t = (int)rows_t;
-    p.tiles_n = (int)((2 * C + 255) / 256);
+    p.tiles_n = (int)((2 * C + ca2::kProjBN - 1) / ca2::kProjBN);
     p.tiles_t = (int)((rows_t + 127) / 128) * p.tiles_n;
     p.tiles_s_frame = (g.hw + 127) / 128;
     p.k_steps = (int)((C + 63) / 64);
@@ -396,10 +396,10 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     ca2::KvProjMaps m;
     std::memset(&m, 0, sizeof(m));
     bool ok = encode_rows_3d(&m.xt, x_t, C, rows_t, 1, C, rows_t * C, 128) &&
-              encode_rows_3d(&m.wt, w_t, C, 2 * C, 1, C, 2 * C * C, 256);
+              encode_rows_3d(&m.wt, w_t, C, 2 * C, 1, C, 2 * C * C, ca2::kProjBN);
     if (ok && n_sp > 0)
         ok = encode_rows_3d(&m.xs, x_s, C, g.hw, (long long)g.batch * n, C, (long long)g.hw * C, 128) &&
-             encode_rows_3d(&m.ws, w_s, C, 2 * C, 1, C, 2 * C * C, 256);
+             encode_rows_3d(&m.ws, w_s, C, 2 * C, 1, C, 2 * C * C, ca2::kProjBN);
     else
         m.xs = m.xt, m.ws = m.wt;    // no spatial tile reads them
     if (!ok) {

@@ -124,6 +124,13 @@ cudaError_t launch_tpe_add(const TpeAddParams &p, cudaStream_t stream);
 // Output tiles of 128 rows x 256 channels over [K | V] (2C channels); temporal tiles first,
 // then spatial tiles.  Rows: temporal (b, s, f) of the token-major chunk input; spatial
 // (s) of one of the chunk's last n_sp frames.
+// Output channels per tile (TMEM columns of the accumulator) and k-steps of 64 input
+// channels in flight.  Measured at C = 1152 (one layer, 2048 + 768 rows): 192 x 5 stages
+// 24.9 us, 128 x 6 stages 27.9 us, 256 x 4 stages 30.4 us -- a deeper ring and 1.8 rather
+// than 1.3 waves of tiles on the 148 SMs.
+constexpr int kProjBN = 192;
+constexpr int kProjStages = 5;
+
 struct KvProjParams {
     __nv_bfloat16 *ring_k, *ring_v;       // this layer's K and V rings [B][HW][H][Pmax][D]
     __nv_bfloat16 *sp_k, *sp_v;           // this layer's spatial cache [P'][B][HW][H][D]
@@ -132,13 +139,13 @@ struct KvProjParams {
     int p_max, slot0;       // ring slot of chunk frame 0
     int n_sp;               // chunk frames stored in the spatial cache (the last n_sp)
     int rows_t;             // B * HW * n
-    int tiles_n;            // ceil(2C / 256)
+    int tiles_n;            // ceil(2C / kProjBN)
     int tiles_t;            // temporal tiles: ceil(rows_t / 128) * tiles_n
     int tiles_s_frame;      // spatial row tiles per frame: ceil(HW / 128)
     int k_steps;            // ceil(C / 64)
 };
 
-// A tiles: boxes of 64 channels x 128 rows (x 1 frame); W tiles: 64 channels x 256 rows;
+// A tiles: boxes of 64 channels x 128 rows (x 1 frame); W tiles: 64 channels x kProjBN rows;
 // all with 128-byte rows and the 128-byte swizzle.  xt, wt: 3-D views with one plane;
 // xs: (channel, token, frame) of the frame-major chunk input.
 struct KvProjMaps {

@@ -8,15 +8,15 @@
 //             ring slot (slot0 + f) mod Pmax of token (b, s) -- the ring's own layout;
 //   spatial : row s of frame f of x_s [B][n][HW][C], f among the chunk's last n_sp frames
 //             -> [K | V] = x_s W_s^T + b_s, stored in spatial-cache frame f - (n - n_sp).
-// The projections never exist as a tensor of their own: each 128-row x 256-channel output
+// The projections never exist as a tensor of their own: each 128-row x 192-channel output
 // tile is accumulated in TMEM and written from registers straight to its cache rows, so
 // the separate cache write (a read and a write of every K and V) disappears.
 //
 // One CTA per output tile; the temporal and spatial tiles share one grid.  Four warps:
-//   warp 0   TMA producer: per 64-channel k-step an A tile (128 rows) and a W tile (256
+//   warp 0   TMA producer: per 64-channel k-step an A tile (128 rows) and a W tile (192
 //            output channels), 128-byte rows with the 128-byte swizzle, kStages deep.
 //   warp 1   MMA issuer (whole warp, one elected lane): per k-step four tcgen05.mma of
-//            M = 128, N = 256, K = 16 into a 256-column fp32 accumulator in TMEM.
+//            M = 128, N = 192, K = 16 into a 192-column fp32 accumulator in TMEM.
 //   all 4    epilogue: warp w reads TMEM lanes 32w..32w+31 (its 32 rows), 32 columns at
 //            a time, adds the bias, rounds to bf16 (nearest, ties to even) and stores
 //            16-byte pieces of 8 channels; a piece never crosses a head because D and C
@@ -38,12 +38,13 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kBM = 128;                                  // rows per tile (TMEM lanes)
-constexpr int kBN = 256;                                  // output channels per tile (TMEM columns)
+constexpr int kBN = kProjBN;                              // output channels per tile (TMEM columns)
 constexpr int kBK = 64;                                   // input channels per k-step (128-byte rows)
-constexpr int kStages = 4;
+constexpr int kStages = kProjStages;
 constexpr uint32_t kATile = kBM * kBK * 2;                // 16 KB
-constexpr uint32_t kWTile = kBN * kBK * 2;                // 32 KB
+constexpr uint32_t kWTile = kBN * kBK * 2;                // 24 KB
 constexpr uint32_t kStageBytes = kATile + kWTile;
+constexpr uint32_t kTmemCols = kBN <= 32 ? 32u : kBN <= 64 ? 64u : kBN <= 128 ? 128u : 256u;   // power of 2
 constexpr uint32_t kSw128 = 2;                            // smem-descriptor layout code: 128-byte swizzle
 constexpr uint32_t kBarBytes = 8u * (2 * kStages + 1) + 16u;   // barriers, abort flag, TMEM address
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024u;   // + base alignment
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
         prefetch_tmap(mw);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32((const void *)tmem_slot), (uint32_t)kBN);
+        tmem_alloc(smem_u32((const void *)tmem_slot), kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)kBN);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
