@@ -337,6 +337,35 @@ def run_ca2(args):
     avg_tpe = ta.elapsed_time(tb) / 1e3 / (5 * NL)
     del gt
 
+    # ---- K/V projection with the cache write fused (a next-row kernel, timed on its own) ----
+    # one launch per block: the cache-writing pass's temporal and spatial K/V projections
+    # (random weights per block, bias included) stored straight into the ring and spatial
+    # cache; 28 launches in a CUDA graph, replayed 5 times.  The queue is full, so 8 frames
+    # are evicted first and committed back afterwards (the same queue length as the step).
+    C = H * D
+    n_sp = min(PS, l)
+    wk = [[(torch.randn((2 * C, C), generator=g, device=dev) * C ** -0.5).to(torch.bfloat16) for _ in range(2)]
+          for _ in range(NL)]
+    bk = [(torch.randn((2 * C,), generator=g, device=dev) * 0.1).to(torch.bfloat16) for _ in range(NL)]
+    cache.evict_for(l)
+    gp = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        gp.capture_begin()
+        for L in range(NL):
+            ca2.ca2_kv_proj_write(h, L, P[L]["tk"], wk[L][0], bk[L], P[L]["sk"], wk[L][1], bk[L], l, cap_sp)
+        gp.capture_end()
+    gp.replay()
+    torch.cuda.synchronize()
+    ta.record(stream)
+    for _ in range(5):
+        gp.replay()
+    tb.record(stream)
+    torch.cuda.synchronize()
+    avg_proj = ta.elapsed_time(tb) / 1e3 / (5 * NL)
+    cache.commit(l)
+    assert ca2.ca2_device_status() == 0
+    del gp, wk, bk
+
     # ---- roofline of each kernel ----
     pk, pk_kind = peaks()
     t_bytes = (2 * PM + 4 * l) * frame_bytes                       # cache K,V + chunk Q,K,V + O
@@ -344,6 +373,7 @@ def run_ca2(args):
     s_flops_self = 4 * D * HW * HW * l * H * B                     # self-repeat mode (own frame once)
     w_bytes = 2 * NL * (2 * l + 2 * PS) * frame_bytes              # read + write of K,V (temporal, spatial)
     tpe_bytes = 2 * l * frame_bytes + l * H * D * 2                 # chunk read + write, n table rows
+    proj_flops = 2 * B * HW * (l + n_sp) * 2 * C * C               # temporal + spatial [K | V] = x W^T
     avg_t = statistics.mean(tp_ms) / 1e3
     avg_sd = statistics.mean(sp_den) / 1e3
     avg_ss = statistics.mean(sp_self) / 1e3
@@ -360,6 +390,10 @@ def run_ca2(args):
         "tpe_add": {"bound": "hbm", "us": avg_tpe * 1e6, "achieved": tpe_bytes / avg_tpe / 1e9,
                     "peak": pk["hbm_gbs"], "unit": "GB/s", "bytes_per_launch": tpe_bytes,
                     "note": "timed apart from the step: 28 launches in a graph, replayed 5 times"},
+        "kv_proj_write": {"bound": "tensor", "us": avg_proj * 1e6, "achieved": proj_flops / avg_proj / 1e12,
+                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "flops_per_launch": proj_flops,
+                          "note": "timed apart from the step (28 launches in a graph, replayed 5 times) "
+                                  "against the burst bf16 peak"},
     }
     for k in kernels.values():
         k["frac"] = k["achieved"] / k["peak"]
