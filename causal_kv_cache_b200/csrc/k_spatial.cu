@@ -16,9 +16,10 @@
 //                not a multiple of 32, padding column D of each landed V tile is set to 1.0
 //                (by warp 3), so the P V product also accumulates the row sum of the
 //                probabilities into O[:, D].
-//   warps 1, 2   MMA issuers of tile A and tile B (one thread each; warp 1 owns the 512
-//                TMEM columns).  A single thread issues about one tcgen05.mma per ~100
-//                cycles whatever the tile width, so each tile has its own issuer.  The
+//   warps 1, 2   MMA issuers of tile A and tile B (the whole warp runs the loop, one
+//                elected lane issues; warp 1 owns the 512 TMEM columns).  A divergent
+//                single thread issued about one tcgen05.mma per ~100 cycles, the whole warp
+//                with warp-uniform operands reaches the tensor rate.  The
 //                tile's next QK^T is issued as soon as its softmax warps have read the
 //                current scores, and its P V product chunk by chunk as the probabilities
 //                land, so the tensor core works while the exponentials run.
@@ -27,11 +28,13 @@
 //                % 4 selects the lane quarter) holding all 128 scores of a block in
 //                registers, so the row max needs no exchange.  The exponential unit
 //                (measured 16 lanes/clock/SM) is the scarce pipe; both tiles' warps share
-//                it, so one warp's stalls are filled by the other's work.  The tiles fill
-//                one shared TMEM probability region in turns, chunk by chunk, each turn
-//                waiting for the P V products of the previous one.  The running max moves
-//                only when it grows by more than 2^8 (O is then rescaled in TMEM).  The
-//                bf16 probabilities are the A operand of the P V product, read from TMEM.
+//                it, so one warp's stalls are filled by the other's work.  Each tile writes
+//                its bf16 probabilities into its own buffer in shared memory (the A operand
+//                of the P V product) and hands a whole block to its issuer with one proxy
+//                fence, so the tiles never wait for each other; at D = 128 they are written
+//                over the tile's scores in TMEM and handed over chunk by chunk.
+//                The running max moves only when it grows by more than 2^8 (O is then
+//                rescaled in TMEM).
 //                Epilogue: O / l -> bf16 rows staged in the tile's spent Q buffer -> one
 //                TMA store of 32 rows per warp.
 //
@@ -106,11 +109,19 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
 __host__ __device__ constexpr int n32(int nkd) { return (nkd + 1) / 2; }
 __host__ __device__ constexpr uint32_t tile_bytes(int nkd) { return n32(nkd) * 8192u; }
 __host__ __device__ constexpr uint32_t tile_slot(int nkd) { return (tile_bytes(nkd) + 1023u) & ~1023u; }
+// Probabilities in shared memory (one 128 x 128 bf16 buffer per tile, four boxes of 32 keys in
+// the same 64-byte-swizzled layout as Q) when the padded head dim is at most 96; at 128 they
+// are written over the tile's own scores in TMEM instead (no room for both buffers).
+__host__ __device__ constexpr bool p_in_smem(int nkd) { return n32(nkd) <= 3; }
+__host__ __device__ constexpr uint32_t p_bytes(int nkd) { return p_in_smem(nkd) ? 2u * 4u * 8192u : 0u; }
 // K and V ring depth: three blocks when it fits in shared memory, else two
-__host__ __device__ constexpr int kv_stages(int nkd) { return 8 * tile_slot(nkd) + 1280u <= 232448u ? 3 : 2; }
+__host__ __device__ constexpr int kv_stages(int nkd)
+{
+    return 8u * tile_slot(nkd) + p_bytes(nkd) + 1536u <= 232448u ? 3 : 2;
+}
 
 struct SmemLayout {
-    uint32_t q0, k0, v0, bars, red, total;
+    uint32_t q0, k0, v0, p0, bars, total;
 };
 
 __host__ __device__ constexpr SmemLayout spatial_layout(int nkd)
@@ -119,31 +130,33 @@ __host__ __device__ constexpr SmemLayout spatial_layout(int nkd)
     L.q0 = 0;                                            // Q of tile A, then tile B
     L.k0 = 2 * tile_slot(nkd);
     L.v0 = L.k0 + kv_stages(nkd) * tile_slot(nkd);
-    L.bars = L.v0 + kv_stages(nkd) * tile_slot(nkd);
-    L.red = L.bars + 512;            // row-max exchange: [2][2][2][128] floats
-    L.total = L.red + 4096 + 1024;   // + slack for the 1024-byte base alignment
+    L.p0 = L.v0 + kv_stages(nkd) * tile_slot(nkd);     // P of tile A, then tile B (32 KB each)
+    L.bars = L.p0 + p_bytes(nkd);
+    L.total = L.bars + 512 + 1024;   // barriers and flags; slack for the 1024-byte base alignment
     return L;
 }
 
-// TMEM columns (512 allocated).  When the padded head dim DP is at most 96 the two tiles
-// keep separate score regions and share one probability region:
-//   S_A [0,128)  S_B [128,256)  P [256,320)  O_A [320,320+DP)  O_B [320+DP,320+2DP)
-// so a tile's next scores can be computed while its probabilities are still being
-// written and read.  With DP = 128 there is no room for that: P is written over the
-// tile's own scores and the next QK^T waits for the P V product.
+// TMEM columns (512 allocated).  With the probabilities in shared memory (padded head dim DP
+// at most 96) TMEM holds each tile's scores and output only:
+//   S_A [0,128)  S_B [128,256)  O_A [256,256+DP)  O_B [256+DP,256+2DP)
+// so a tile's next scores can be computed while its probabilities are still being written and
+// read.  With DP = 128, P is written over the tile's own scores and the next QK^T waits for
+// the P V product.
 template <int NB32>
 struct TmemMap {
     static constexpr int DP = 32 * NB32;
-    static constexpr bool kSharedP = NB32 <= 3;
+    static constexpr bool kPSmem = NB32 <= 3;
     __host__ __device__ static constexpr uint32_t s(int X) { return (uint32_t)X * 128u; }
-    __host__ __device__ static constexpr uint32_t p(int X) { return kSharedP ? 256u : (uint32_t)X * 128u; }
+    __host__ __device__ static constexpr uint32_t p(int X) { return (uint32_t)X * 128u; }   // P over S (DP = 128)
     __host__ __device__ static constexpr uint32_t o(int X)
     {
-        return kSharedP ? 320u + (uint32_t)(X * DP) : 256u + (uint32_t)X * 128u;
+        return kPSmem ? 256u + (uint32_t)(X * DP) : 256u + (uint32_t)X * 128u;
     }
 };
 static_assert(TmemMap<3>::o(1) + 96 <= kTmemCols, "TMEM map overflows");
 static_assert(TmemMap<4>::o(1) + 128 <= kTmemCols, "TMEM map overflows");
+static_assert(TmemMap<3>::kPSmem == p_in_smem(5) && !TmemMap<4>::kPSmem, "P placement mismatch");
+static_assert(8 * 34 + 16 <= 512, "barrier region overflows");
 
 constexpr int kChunks = 4;            // probability chunks per block: 32 keys = 16 P columns each
 constexpr int kSoftmaxWarp0 = 4;      // warps 4..7 tile A, 8..11 tile B
@@ -158,11 +171,12 @@ enum : int {
     B_VEMPTY = 13,    // 3: both tiles' P V of the block are done (2 commits)
     B_SFULL = 16,     // 2 [X]: scores in TMEM
     B_SFREE = 18,     // 2 [X]: every softmax warp of the tile has read the scores (4 warps)
-    B_PFULL = 20,     // 8 [X][c]: probability chunk in TMEM (4 warps)
-    B_PFREE = 28,     // 4 [c]: the P V products reading the shared chunk are done
-    B_ODONE = 32,     // 2 [X]: P V of the block done (all prior products of the tile)
-    B_FIN = 34,       // 2 [X]: every product the tile's issuer launched is done
-    B_COUNT = 36
+    B_PFULL = 20,     // 8 [X][c]: probabilities written (4 warps): per chunk in TMEM, or the
+                      //           whole block in shared memory ([X][0] only)
+    B_PFREE = 28,     // 2 [X]: the P V product reading P_X in shared memory is done
+    B_ODONE = 30,     // 2 [X]: P V of the block done (all prior products of the tile)
+    B_FIN = 32,       // 2 [X]: every product the tile's issuer launched is done
+    B_COUNT = 34
 };
 static_assert(8 * B_COUNT + 12 <= 512, "barrier area");
 
@@ -179,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     constexpr int DP = 32 * NB32;                // P V width (padded head dim)
     constexpr uint32_t TB = tile_slot(NKD);
     using TM = TmemMap<NB32>;
-    constexpr bool kSharedP = TM::kSharedP;
+    constexpr bool kPSmem = TM::kPSmem;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;  // 1024-aligned base for the swizzled tiles
     uint8_t *sgen = smem_raw + (sb - raw);
@@ -237,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             mbar_init(bar(B_FIN + i), 1);
         }
         for (int i = 0; i < 2 * kChunks; ++i) mbar_init(bar(B_PFULL + i), 4);
-        for (int i = 0; i < kChunks; ++i) mbar_init(bar(B_PFREE + i), 1);
+        for (int i = 0; i < 2; ++i) mbar_init(bar(B_PFREE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm.q);
@@ -325,6 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         const uint64_t dq = sdesc(sb + L.q0 + X * TB, 16, 512, kSw64);
         const uint64_t dk0 = sdesc(sb + L.k0, 16, 512, kSw64);
         const uint64_t dv0 = sdesc(sb + L.v0, 8192, 512, kSw64);
+        // P_X in shared memory: K-major like Q (keys along the swizzled rows)
+        const uint64_t dp = sdesc(sb + L.p0 + (uint32_t)X * 32768u, 16, 512, kSw64);
         auto koff = [](int kk) -> uint64_t { return (uint64_t)(((kk >> 1) * 8192 + (kk & 1) * 32) >> 4); };
         const uint32_t s_x = tm_u + TM::s(X), p_x = tm_u + TM::p(X), o_x = tm_u + TM::o(X);
         // S_X = Q_X K(j)^T; the commits release the scores to the softmax warps and
@@ -337,15 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             tc_commit_w(bar(B_SFULL + X));
             tc_commit_w(bar(B_KEMPTY + j % NS));
         };
-        // O_X (+)= P chunk c V(j): P holds two bf16 per column, 8 columns per 16 keys;
-        // chunk c is columns 16c..16c+15 (keys 32c..32c+31), k-steps 2c and 2c+1
+        // O_X (+)= P chunk c V(j), keys 32c..32c+31 = k-steps 2c and 2c+1: from P_X's box c
+        // in shared memory, or (P over S) from TMEM columns 16c..16c+15 (two bf16 per column)
         auto issue_pv = [&](int j, int c) {
             const uint64_t bv = dv0 + (uint64_t)(((j % NS) * TB) >> 4);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int kk = 2 * c + e;
-                tc_mma_ts_w(o_x, p_x + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
-                            (j > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (kPSmem)
+                    tc_mma_ss_w(o_x, dp + koff(kk), bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                else
+                    tc_mma_ts_w(o_x, p_x + 8 * kk, bv + (uint64_t)((kk * 1024) >> 4), idesc_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
             }
         };
         bool ok = warp_wait(bar(B_QFULL), 0, 211, abort_flag) && warp_wait(bar(B_KFULL), 0, 212, abort_flag);
@@ -354,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             issue_qk(0);
         }
         for (int j = 0; ok && j < NB; ++j) {
-            if (kSharedP && j + 1 < NB) {
+            if (kPSmem && j + 1 < NB) {
                 // the tile's score region is free once its softmax warps have read S(j):
                 // compute S(j+1) while they exponentiate
                 const int j1 = j + 1;
@@ -366,16 +386,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             }
             if (!warp_wait(bar(B_VREADY + j % NS), (j / NS) & 1, 215, abort_flag)) break;
             bool okc = true;
-            for (int c = 0; c < kChunks; ++c) {
-                if (!warp_wait(bar(B_PFULL + kChunks * X + c), j & 1, 216, abort_flag)) { okc = false; break; }
-                tc_fence_after();
-                issue_pv(j, c);
-                if (kSharedP) tc_commit_w(bar(B_PFREE + c));
+            if constexpr (kPSmem) {
+                // the whole block's probabilities at once (one proxy fence per softmax warp)
+                okc = warp_wait(bar(B_PFULL + kChunks * X), j & 1, 216, abort_flag);
+                if (okc) {
+                    tc_fence_after();
+                    for (int c = 0; c < kChunks; ++c) issue_pv(j, c);
+                    tc_commit_w(bar(B_PFREE + X));
+                }
+            } else {
+                for (int c = 0; c < kChunks; ++c) {
+                    if (!warp_wait(bar(B_PFULL + kChunks * X + c), j & 1, 216, abort_flag)) { okc = false; break; }
+                    tc_fence_after();
+                    issue_pv(j, c);
+                }
             }
             if (!okc) break;
             tc_commit_w(bar(B_ODONE + X));
             tc_commit_w(bar(B_VEMPTY + j % NS));
-            if (!kSharedP && j + 1 < NB) {
+            if (!kPSmem && j + 1 < NB) {
                 // P was written over S: the next scores follow the P V product
                 const int j1 = j + 1;
                 if (!warp_wait(bar(B_KFULL + j1 % NS), (j1 / NS) & 1, 214, abort_flag)) break;
@@ -425,6 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         const uint32_t s_col = tmem + lane_bits + TM::s(X);
         const uint32_t p_col = tmem + lane_bits + TM::p(X);
         const uint32_t o_col = tmem + lane_bits + TM::o(X);
+        // this row of P_X in shared memory (box c adds c * 8 KB): 8-row groups 512 B apart,
+        // 64-byte rows whose four 16-byte pieces are swizzled by (row >> 1) & 3
+        const uint32_t p_row = sb + L.p0 + (uint32_t)X * 32768u + (uint32_t)(row >> 3) * 512u + (uint32_t)(row & 7) * 64u;
+        const uint32_t p_swz = (uint32_t)((row >> 1) & 3);
         const float neg_inf = __int_as_float(0xff800000);
         const float scale = p.scale_log2;
         float m_used = neg_inf;     // max (log2 units) the probabilities are taken against
@@ -478,11 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 }
             }
             l_sum *= alpha;
-            // probabilities from the registers as bf16 pairs (keys 32c.. -> P columns
-            // 16c..), handed to the issuer one chunk at a time; a chunk's store completes
-            // while the next chunk's exponentials run
+            // probabilities from the registers as bf16 pairs, handed to the issuer one chunk
+            // of 32 keys at a time
             const float neg_m = -m_used;
-            const int use = 2 * j + X;    // turn of this tile on the shared P region
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
                 // all 32 exponentials of the chunk first, so that a warp keeps many in
@@ -503,25 +534,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                     if (!ones_col) ls += bf16_lo(w[i]) + bf16_hi(w[i]);
                 }
                 l_sum += ls;
-                if (c > 0) {
-                    // the previous chunk has landed: hand it over
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + c - 1));
+                if constexpr (kPSmem) {
+                    // keys 32c.. -> box c of P_X; this tile's P V of the previous block must be
+                    // done reading P_X before its first chunk is overwritten
+                    if (c == 0 && j > 0 && !warp_wait(bar(B_PFREE + X), (j - 1) & 1, 229, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a = p_row + (uint32_t)c * 8192u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a + (((uint32_t)q ^ p_swz) << 4)),
+                                     "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                                     : "memory");
+                    if (c == kChunks - 1) {
+                        // one proxy fence for the block (a fence per chunk measured 29.5 us
+                        // per launch against 24.3), then the block goes to the issuer
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X));
+                    }
+                } else {
+                    // P over S (keys 32c.. -> TMEM columns 16c..): a chunk's store completes
+                    // while the next chunk's exponentials run, then it is handed over
+                    if (c > 0) {
+                        tmem_st_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + c - 1));
+                    }
+                    tmem_st16(p_col + (uint32_t)(16 * c), w);
                 }
-                if (kSharedP && use > 0) {
-                    // the other tile's P V products must be done reading this chunk
-                    if (!warp_wait(bar(B_PFREE + c), (use - 1) & 1, 229, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                }
-                tmem_st16(p_col + (uint32_t)(16 * c), w);
             }
             if (!ok) break;
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + kChunks - 1));
+            if constexpr (!kPSmem) {
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_PFULL + kChunks * X + kChunks - 1));
+            }
         }
         // ---- epilogue: O / l -> bf16 rows staged in the tile's (now unused) Q buffer,
         //      then one TMA store of the warp's 32 rows -----------------------------------
