@@ -391,6 +391,7 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     p.k_steps = (int)((C + 63) / 64);
     const long long tiles_s = (long long)g.batch * n_sp * p.tiles_s_frame * p.tiles_n;
     if (p.tiles_t + tiles_s >= (1ll << 31)) return CA2_ERR_SHAPE;
+    p.total_tiles = (int)(p.tiles_t + tiles_s);
 
     // x_t: [B*HW*n][C]; x_s: (C, HW, B*n frames); W: [2C][C] (output channel rows)
     ca2::KvProjMaps m;
@@ -406,7 +407,11 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
         g_last_cuda_error = "tensor-map encoding failed";
         return CA2_ERR_CUDA;
     }
-    return cuda_status(ca2::launch_kv_proj(m, p, (int)(p.tiles_t + tiles_s), static_cast<cudaStream_t>(stream)));
+    // persistent: one CTA per SM (or per tile when there are fewer tiles)
+    const int sms = sm_count();
+    if (sms <= 0) return CA2_ERR_CUDA;
+    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    return cuda_status(ca2::launch_kv_proj(m, p, grid, static_cast<cudaStream_t>(stream)));
 }
 
 int ca2_cache_commit(ca2_cache *c, int n)

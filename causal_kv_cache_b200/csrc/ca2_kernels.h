@@ -143,6 +143,7 @@ struct KvProjParams {
     int tiles_t;            // temporal tiles: ceil(rows_t / 128) * tiles_n
     int tiles_s_frame;      // spatial row tiles per frame: ceil(HW / 128)
     int k_steps;            // ceil(C / 64)
+    int total_tiles;        // temporal + spatial tiles (the persistent grid walks them)
 };
 
 // A tiles: boxes of 64 channels x 128 rows (x 1 frame); W tiles: 64 channels x kProjBN rows;

@@ -12,18 +12,22 @@
 // tile is accumulated in TMEM and written from registers straight to its cache rows, so
 // the separate cache write (a read and a write of every K and V) disappears.
 //
-// One CTA per output tile; the temporal and spatial tiles share one grid.  Four warps:
-//   warp 0   TMA producer: per 64-channel k-step an A tile (128 rows) and a W tile (192
-//            output channels), 128-byte rows with the 128-byte swizzle, kStages deep.
-//   warp 1   MMA issuer (whole warp, one elected lane): per k-step four tcgen05.mma of
-//            M = 128, N = 192, K = 16 into a 192-column fp32 accumulator in TMEM.
-//   all 4    epilogue: warp w reads TMEM lanes 32w..32w+31 (its 32 rows), 32 columns at
-//            a time, adds the bias, rounds to bf16 (nearest, ties to even) and stores
-//            16-byte pieces of 8 channels; a piece never crosses a head because D and C
-//            are multiples of 8.
+// Persistent: one CTA per SM walks the output tiles (temporal tiles first, then spatial)
+// with a stride of the grid.  Six warps:
+//   warp 0     TMA producer: per 64-channel k-step an A tile (128 rows) and a W tile (192
+//              output channels), 128-byte rows with the 128-byte swizzle, into a ring of
+//              kStages slots that runs on across tiles.
+//   warp 1     MMA issuer (whole warp, one elected lane): per k-step four tcgen05.mma of
+//              M = 128, N = 192, K = 16, into one of two fp32 TMEM accumulators (columns
+//              0 and 256), alternating by tile.
+//   warps 2-5  epilogue of the other accumulator while the next tile accumulates: warp w
+//              reads TMEM lanes 32 (w % 4).. (its rows), 32 columns at a time, adds the
+//              bias, rounds to bf16 (nearest, ties to even) and stores 16-byte pieces of 8
+//              channels; a piece never crosses a head because D and C are multiples of 8.
 // Channels past C in a k-step, rows past the end and output channels past 2C are
 // zero-filled by the TMA unit; the epilogue skips rows and channels that do not exist.
-// Every mbarrier wait is bounded; a timeout is recorded in the library status word.
+// Every mbarrier wait is bounded; a timeout is recorded in the library status word and all
+// roles wind down (issued copies land, issued MMAs complete, TMEM is freed).
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -36,18 +40,24 @@ namespace ca2 {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;
 constexpr int kBM = 128;                                  // rows per tile (TMEM lanes)
-constexpr int kBN = kProjBN;                              // output channels per tile (TMEM columns)
+constexpr int kBN = kProjBN;                              // output channels per tile
 constexpr int kBK = 64;                                   // input channels per k-step (128-byte rows)
 constexpr int kStages = kProjStages;
+constexpr uint32_t kAccStride = 256;                      // TMEM columns between the two accumulators
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kATile = kBM * kBK * 2;                // 16 KB
 constexpr uint32_t kWTile = kBN * kBK * 2;                // 24 KB
 constexpr uint32_t kStageBytes = kATile + kWTile;
-constexpr uint32_t kTmemCols = kBN <= 32 ? 32u : kBN <= 64 ? 64u : kBN <= 128 ? 128u : 256u;   // power of 2
 constexpr uint32_t kSw128 = 2;                            // smem-descriptor layout code: 128-byte swizzle
-constexpr uint32_t kBarBytes = 8u * (2 * kStages + 1) + 16u;   // barriers, abort flag, TMEM address
+// barriers: full[S], empty[S], acc_full[2], acc_empty[2], fin; then the abort flag and the
+// TMEM address
+constexpr int kBars = 2 * kStages + 5;
+constexpr uint32_t kBarBytes = 8u * kBars + 16u;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024u;   // + base alignment
+static_assert(kBN <= (int)kAccStride && kAccStride + kBN <= kTmemCols, "accumulators overflow TMEM");
+static_assert(kSmemBytes <= 232448u, "shared memory overflows");
 
 // the bias of 8 consecutive channels (16 bytes), or zeros
 __device__ __forceinline__ void bias8(const __nv_bfloat16 *b, int ch, float (&f)[8])
@@ -62,6 +72,31 @@ __device__ __forceinline__ void bias8(const __nv_bfloat16 *b, int ch, float (&f)
     }
 }
 
+// one output tile: problem, row tile, channel tile, and for a spatial tile the video and
+// the spatial-cache frame (plane = frame of x_s read)
+struct Tile {
+    bool spatial;
+    int tn, tm, jsp, vid, plane;
+};
+
+__device__ __forceinline__ Tile decode_tile(const KvProjParams &p, int t)
+{
+    Tile d{};
+    d.spatial = t >= p.tiles_t;
+    if (d.spatial) t -= p.tiles_t;
+    d.tn = t % p.tiles_n;
+    t /= p.tiles_n;
+    d.tm = t;
+    if (d.spatial) {
+        d.tm = t % p.tiles_s_frame;
+        t /= p.tiles_s_frame;
+        d.jsp = t % p.n_sp;
+        d.vid = t / p.n_sp;
+        d.plane = d.vid * p.n + (p.n - p.n_sp) + d.jsp;
+    }
+    return d;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__ KvProjMaps tm, const KvProjParams p)
@@ -73,39 +108,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
     const uint32_t bars = sb + kStages * kStageBytes;
     auto full_bar = [&](int s) { return bars + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return bars + 8u * (uint32_t)(kStages + s); };
-    const uint32_t acc_bar = bars + 8u * (uint32_t)(2 * kStages);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + kStages * kStageBytes + 8 * (2 * kStages + 1));
-    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + kStages * kStageBytes + 8 * (2 * kStages + 1) + 8);
+    auto acc_full = [&](int a) { return bars + 8u * (uint32_t)(2 * kStages + a); };
+    auto acc_empty = [&](int a) { return bars + 8u * (uint32_t)(2 * kStages + 2 + a); };
+    const uint32_t fin_bar = bars + 8u * (uint32_t)(2 * kStages + 4);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sgen + kStages * kStageBytes + 8 * kBars);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sgen + kStages * kStageBytes + 8 * kBars + 8);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // tile -> problem, row tile, channel tile (and for a spatial tile: video, frame)
-    int t = blockIdx.x;
-    const bool spatial = t >= p.tiles_t;
-    if (spatial) t -= p.tiles_t;
-    const int tn = t % p.tiles_n;
-    t /= p.tiles_n;
-    int tm_row = t, jsp = 0, vid = 0, plane = 0;
-    if (spatial) {
-        tm_row = t % p.tiles_s_frame;
-        t /= p.tiles_s_frame;
-        jsp = t % p.n_sp;                                 // spatial-cache frame
-        vid = t / p.n_sp;
-        plane = vid * p.n + (p.n - p.n_sp) + jsp;         // frame of x_s read
-    }
-    const CUtensorMap *ma = spatial ? &tm.xs : &tm.xt;
-    const CUtensorMap *mw = spatial ? &tm.ws : &tm.wt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(acc_bar, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(acc_full(a), 1);
+            mbar_init(acc_empty(a), 4);                   // the four epilogue warps
+        }
+        mbar_init(fin_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(ma);
-        prefetch_tmap(mw);
+        prefetch_tmap(&tm.xt);
+        prefetch_tmap(&tm.wt);
+        prefetch_tmap(&tm.xs);
+        prefetch_tmap(&tm.ws);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32((const void *)tmem_slot), kTmemCols);
@@ -121,102 +147,126 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
 
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
-        int issued = -1;
-        for (int ks = 0; ks < p.k_steps; ++ks) {
-            const int s = ks % kStages;
-            if (ks >= kStages && !warp_wait(empty_bar(s), ((ks / kStages) - 1) & 1, 301, abort_flag)) break;
-            if (lane == 0) {
-                const uint32_t a = sb + (uint32_t)s * kStageBytes;
-                mbar_expect_tx(full_bar(s), kStageBytes);
-                tma_load_3d(a, ma, ks * kBK, tm_row * kBM, plane, full_bar(s));
-                tma_load_3d(a + kATile, mw, ks * kBK, tn * kBN, 0, full_bar(s));
+        int g = 0;                                        // k-steps issued by this CTA
+        for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+            const Tile d = decode_tile(p, t);
+            const CUtensorMap *ma = d.spatial ? &tm.xs : &tm.xt;
+            const CUtensorMap *mw = d.spatial ? &tm.ws : &tm.wt;
+            bool ok = true;
+            for (int ks = 0; ks < p.k_steps; ++ks, ++g) {
+                const int s = g % kStages;
+                if (g >= kStages && !warp_wait(empty_bar(s), ((g / kStages) - 1) & 1, 301, abort_flag)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t a = sb + (uint32_t)s * kStageBytes;
+                    mbar_expect_tx(full_bar(s), kStageBytes);
+                    tma_load_3d(a, ma, ks * kBK, d.tm * kBM, d.plane, full_bar(s));
+                    tma_load_3d(a + kATile, mw, ks * kBK, d.tn * kBN, 0, full_bar(s));
+                }
+                __syncwarp();
             }
-            issued = ks;
-            __syncwarp();
+            if (!ok) break;
         }
         // wind-down after an abort: the issued loads land before the CTA exits
         if (lane == 0 && *abort_flag)
-            for (int ks = issued; ks >= 0 && ks > issued - kStages; --ks)
-                mbar_wait(full_bar(ks % kStages), (ks / kStages) & 1, 0, nullptr, 2000000ull);
+            for (int k = g - 1; k >= 0 && k >= g - kStages; --k)
+                mbar_wait(full_bar(k % kStages), (k / kStages) & 1, 0, nullptr, 2000000ull);
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
         // K-major operands with the 128-byte swizzle: 8-row groups 1024 B apart; the k-step
         // kk of 16 channels starts 32 B further into each 128-byte row.
         constexpr uint32_t idesc = idesc_bf16(kBM, kBN, false, false);
         const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
-        for (int ks = 0; ks < p.k_steps; ++ks) {
-            const int s = ks % kStages;
-            if (!warp_wait(full_bar(s), (ks / kStages) & 1, 302, abort_flag)) break;
+        int g = 0, i = 0;                                 // k-steps and tiles of this CTA
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x, ++i) {
+            const int acc = i & 1;
+            // the epilogue of the tile that last used this accumulator is done with it
+            if (i >= 2 && !warp_wait(acc_empty(acc), ((i >> 1) - 1) & 1, 304, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t a = sb + (uint32_t)s * kStageBytes;
-            const uint64_t da = sdesc(a, 16, 1024, kSw128);
-            const uint64_t dw = sdesc(a + kATile, 16, 1024, kSw128);
+            const uint32_t d_tmem = tm_u + (uint32_t)acc * kAccStride;
+            for (int ks = 0; ks < p.k_steps; ++ks, ++g) {
+                const int s = g % kStages;
+                if (!warp_wait(full_bar(s), (g / kStages) & 1, 302, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a = sb + (uint32_t)s * kStageBytes;
+                const uint64_t da = sdesc(a, 16, 1024, kSw128);
+                const uint64_t dw = sdesc(a + kATile, 16, 1024, kSw128);
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-                tc_mma_ss_w(tm_u, da + (uint64_t)(2 * kk), dw + (uint64_t)(2 * kk), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-            tc_commit_w(empty_bar(s));
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    tc_mma_ss_w(d_tmem, da + (uint64_t)(2 * kk), dw + (uint64_t)(2 * kk), idesc,
+                                (ks > 0 || kk > 0) ? 1u : 0u);
+                tc_commit_w(empty_bar(s));
+            }
+            if (ok) tc_commit_w(acc_full(acc));
         }
-        // fires once every issued MMA has completed (after an abort too); this warp frees
-        // TMEM, so it waits for that itself, bounded and regardless of the abort flag
-        tc_commit_w(acc_bar);
-        mbar_wait(acc_bar, 0, 0, nullptr, 2000000ull);
+        // every issued MMA completes before TMEM is freed (bounded, regardless of the abort)
+        tc_commit_w(fin_bar);
+        mbar_wait(fin_bar, 0, 0, nullptr, 2000000ull);
         __syncwarp();
-    }
-
-    // ------------------------------- epilogue (all warps) ---------------------------------
-    __syncwarp();
-    const bool acc_ok = warp_wait(acc_bar, 0, 303, abort_flag);
-    if (acc_ok && !*abort_flag) {
-        tc_fence_after();
-        const int r = warp * 32 + lane;                   // row of the tile = TMEM lane
-        // row -> element offset of the row's (h = 0, d = 0) in its cache, and the stride
-        // between consecutive heads
-        long long base = -1;
-        long long head_stride = 0;
-        if (!spatial) {
-            const int m = tm_row * kBM + r;
-            if (m < p.rows_t) {
-                const int f = m % p.n;
-                const long long bs = m / p.n;             // b * HW + s
-                const int slot = (p.slot0 + f) % p.p_max;
-                base = (bs * p.H * p.p_max + slot) * (long long)p.D;
-                head_stride = (long long)p.p_max * p.D;
+    } else {
+        // ------------------------------- epilogue (warps 2-5) --------------------------
+        const int quarter = warp & 3;                     // TMEM lanes 32 * quarter ..
+        const int r = quarter * 32 + lane;                // row of the tile = TMEM lane
+        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        int i = 0;
+        for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++i) {
+            const int acc = i & 1;
+            if (!warp_wait(acc_full(acc), (i >> 1) & 1, 303, abort_flag)) break;
+            tc_fence_after();
+            const Tile d = decode_tile(p, t);
+            // row -> element offset of the row's (h = 0, d = 0) in its cache, and the stride
+            // between consecutive heads
+            long long base = -1;
+            long long head_stride = 0;
+            if (!d.spatial) {
+                const int m = d.tm * kBM + r;
+                if (m < p.rows_t) {
+                    const int f = m % p.n;
+                    const long long bs = m / p.n;         // b * HW + s
+                    const int slot = (p.slot0 + f) % p.p_max;
+                    base = (bs * p.H * p.p_max + slot) * (long long)p.D;
+                    head_stride = (long long)p.p_max * p.D;
+                }
+            } else {
+                const int s = d.tm * kBM + r;
+                if (s < p.HW) {
+                    base = (((long long)d.jsp * p.B + d.vid) * p.HW + s) * (long long)p.H * p.D;
+                    head_stride = p.D;
+                }
             }
-        } else {
-            const int s = tm_row * kBM + r;
-            if (s < p.HW) {
-                base = (((long long)jsp * p.B + vid) * p.HW + s) * (long long)p.H * p.D;
-                head_stride = p.D;
-            }
-        }
-        const __nv_bfloat16 *bias = spatial ? p.bias_s : p.bias_t;
-        __nv_bfloat16 *dst_k = spatial ? p.sp_k : p.ring_k;
-        __nv_bfloat16 *dst_v = spatial ? p.sp_v : p.ring_v;
-        const uint32_t lane_bits = (uint32_t)(warp * 32) << 16;
-        for (int c0 = 0; c0 < kBN; c0 += 32) {
-            const int n0 = tn * kBN + c0;
-            if (n0 >= 2 * p.C) break;                     // warp-uniform
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_bits + (uint32_t)c0, v);
-            if (base < 0) continue;
+            const __nv_bfloat16 *bias = d.spatial ? p.bias_s : p.bias_t;
+            __nv_bfloat16 *dst_k = d.spatial ? p.sp_k : p.ring_k;
+            __nv_bfloat16 *dst_v = d.spatial ? p.sp_v : p.ring_v;
+            const uint32_t acc_cols = tmem + lane_bits + (uint32_t)acc * kAccStride;
+            for (int c0 = 0; c0 < kBN; c0 += 32) {
+                const int n0 = d.tn * kBN + c0;
+                if (n0 >= 2 * p.C) break;                 // warp-uniform
+                uint32_t v[32];
+                tmem_ld32(acc_cols + (uint32_t)c0, v);
+                if (base < 0) continue;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int ch = n0 + 8 * q;
-                if (ch >= 2 * p.C) break;
-                const int kv = ch >= p.C ? 1 : 0;
-                const int rem = ch - kv * p.C;
-                const int h = rem / p.D;
-                const int d = rem - h * p.D;
-                float b8[8];
-                bias8(bias, ch, b8);
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) + b8[0], __uint_as_float(v[8 * q + 1]) + b8[1]);
-                w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + b8[2], __uint_as_float(v[8 * q + 3]) + b8[3]);
-                w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) + b8[4], __uint_as_float(v[8 * q + 5]) + b8[5]);
-                w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) + b8[6], __uint_as_float(v[8 * q + 7]) + b8[7]);
-                __nv_bfloat16 *dst = (kv ? dst_v : dst_k) + base + (long long)h * head_stride + d;
-                *reinterpret_cast<uint4 *>(dst) = w;
+                for (int q = 0; q < 4; ++q) {
+                    const int ch = n0 + 8 * q;
+                    if (ch >= 2 * p.C) break;
+                    const int kv = ch >= p.C ? 1 : 0;
+                    const int rem = ch - kv * p.C;
+                    const int h = rem / p.D;
+                    const int dd = rem - h * p.D;
+                    float b8[8];
+                    bias8(bias, ch, b8);
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) + b8[0], __uint_as_float(v[8 * q + 1]) + b8[1]);
+                    w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + b8[2], __uint_as_float(v[8 * q + 3]) + b8[3]);
+                    w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) + b8[4], __uint_as_float(v[8 * q + 5]) + b8[5]);
+                    w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) + b8[6], __uint_as_float(v[8 * q + 7]) + b8[7]);
+                    __nv_bfloat16 *dst = (kv ? dst_v : dst_k) + base + (long long)h * head_stride + dd;
+                    *reinterpret_cast<uint4 *>(dst) = w;
+                }
             }
+            // the accumulator may take the tile after next
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(acc));
         }
     }
     tc_fence_before();
