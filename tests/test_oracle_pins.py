@@ -206,23 +206,60 @@ def _bf16_bits(vals):
     return (f.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def test_kv_projection_matches_brute_force_loops():
+def _projection_matches_loops(proj) -> bool:
     """Y[r][o] = sum_i x[r][i] w[o][i] + b[o] written out as loops on a tiny case (integer
-    values: exact in any order); K is output channels 0..C-1, V channels C..2C-1.  A
-    transposed weight, a swapped K/V half or a dropped bias fails it."""
+    values: exact in any order); K is output channels 0..C-1, V channels C..2C-1."""
     rng = np.random.default_rng(5)
     rows, C = 3, 4
     x = rng.integers(-4, 5, size=(rows, C))
     w = rng.integers(-3, 4, size=(2 * C, C))
     b = rng.integers(-8, 9, size=(2 * C,))
-    k, v = oracle.kv_projection(_bf16_bits(x), _bf16_bits(w), _bf16_bits(b))
+    try:
+        k, v = proj(_bf16_bits(x), _bf16_bits(w), _bf16_bits(b))
+    except Exception:
+        return False
     for r in range(rows):
         for o in range(2 * C):
             acc = float(b[o])
             for i in range(C):
                 acc += float(x[r][i]) * float(w[o][i])
             got = k[r][o] if o < C else v[r][o - C]
-            assert got == acc, (r, o, got, acc)
+            if got != acc:
+                return False
+    return True
+
+
+def test_kv_projection_matches_brute_force_loops():
+    """The oracle's projection against the written-out loops."""
+    assert _projection_matches_loops(oracle.kv_projection)
+
+
+def test_kv_projection_planted_mistakes_are_caught():
+    """Plausible mistakes in a projection -- K and V halves swapped, the bias dropped, the
+    weight read transposed, an input channel off by one -- each fail the loop pin."""
+    f64 = lambda a: (np.asarray(a).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    def swapped(x, w, b):
+        k, v = oracle.kv_projection(x, w, b)
+        return v, k
+
+    def no_bias(x, w, b):
+        return oracle.kv_projection(x, w, None)
+
+    def transposed(x, w, b):
+        y = f64(x) @ f64(w)[: f64(x).shape[1]]        # w's first C rows as a C x C matrix
+        y = np.concatenate([y, y], axis=1) + f64(b)[None, :]
+        C = f64(x).shape[1]
+        return y[:, :C], y[:, C:]
+
+    def shifted(x, w, b):
+        xs = np.roll(f64(x), 1, axis=1)
+        y = xs @ f64(w).T + f64(b)[None, :]
+        C = xs.shape[1]
+        return y[:, :C], y[:, C:]
+
+    for bad in (swapped, no_bias, transposed, shifted):
+        assert not _projection_matches_loops(bad), bad.__name__
 
 
 def test_kv_projection_identity_and_bias_only():
