@@ -94,7 +94,7 @@ class Generator:
     """Counter-free, order-defined generator: numpy PCG64 seeded once, draws in call order.
 
     Every tensor is returned as raw bf16 bits (np.uint16) in the caller layout
-    [B][n][HW][H][D] (token-major, heads then head dim contiguous).
+    [B][n][HW][H][D] (frame-major: video, frame, token, then heads and head dim contiguous).
     """
 
     def __init__(self, wl: Workload, seed: int = 0):

@@ -17,7 +17,8 @@ from typing import List, Optional, Sequence, Tuple
 
 __all__ = [
     "Ca2Error", "ca2_config", "load_library", "LIBRARY_PATH",
-    "ca2_cache_bytes", "ca2_cache_init", "ca2_cache_destroy", "ca2_cache_evict",
+    "ca2_cache_bytes", "ca2_cache_init", "ca2_cache_destroy", "ca2_cache_evict", "ca2_cache_evict_for",
+    "ca2_cache_config", "ca2_cache_layer_offsets",
     "ca2_cache_write", "ca2_kv_proj_write", "ca2_cache_commit", "ca2_temporal_attn", "ca2_spatial_prefix_attn",
     "ca2_tpe_indices", "ca2_tpe_add",
     "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string",
@@ -29,7 +30,7 @@ LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libca2.
 
 STATUS = {
     0: "CA2_OK", -1: "CA2_ERR_ARG", -2: "CA2_ERR_SHAPE", -3: "CA2_ERR_CAPACITY",
-    -4: "CA2_ERR_ALIGN", -5: "CA2_ERR_CUDA", -6: "CA2_ERR_TIMEOUT",
+    -4: "CA2_ERR_ALIGN", -5: "CA2_ERR_CUDA", -6: "CA2_ERR_TIMEOUT", -7: "CA2_ERR_RANGE",
 }
 
 
@@ -50,6 +51,7 @@ class ca2_config(ctypes.Structure):
         ("n_layers", ctypes.c_int), ("batch", ctypes.c_int), ("hw", ctypes.c_int),
         ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("chunk_len", ctypes.c_int),
         ("p_max", ctypes.c_int), ("p_spatial", ctypes.c_int), ("tpe_len", ctypes.c_int),
+        ("row_pitch", ctypes.c_int),
     ]
 
 
@@ -76,6 +78,9 @@ def load_library(path: Optional[str] = None):
         "ca2_cache_init": ([cfgp, vp, sz, vp, sz, ctypes.POINTER(vp)], i),
         "ca2_cache_destroy": ([vp], i),
         "ca2_cache_evict": ([vp, i], i),
+        "ca2_cache_evict_for": ([vp, i, ctypes.POINTER(i)], i),
+        "ca2_cache_config": ([vp, cfgp], i),
+        "ca2_cache_layer_offsets": ([vp, i, i, ctypes.POINTER(sz), ctypes.POINTER(sz)], i),
         "ca2_cache_write": ([vp, pp, pp, pp, pp, i, vp], i),
         "ca2_kv_proj_write": ([vp, i, vp, vp, vp, vp, vp, vp, i, vp], i),
         "ca2_cache_commit": ([vp, i], i),
@@ -175,6 +180,25 @@ def ca2_cache_evict(handle, n_frames: int) -> None:
     _check(load_library().ca2_cache_evict(handle, int(n_frames)), "ca2_cache_evict")
 
 
+def ca2_cache_evict_for(handle, n_new: int) -> int:
+    e = ctypes.c_int(0)
+    _check(load_library().ca2_cache_evict_for(handle, int(n_new), ctypes.byref(e)), "ca2_cache_evict_for")
+    return e.value
+
+
+def ca2_cache_config(handle) -> ca2_config:
+    c = ca2_config()
+    _check(load_library().ca2_cache_config(handle, ctypes.byref(c)), "ca2_cache_config")
+    return c
+
+
+def ca2_cache_layer_offsets(handle, layer: int, kv: int) -> Tuple[int, int]:
+    t, s_ = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(load_library().ca2_cache_layer_offsets(handle, int(layer), int(kv), ctypes.byref(t), ctypes.byref(s_)),
+           "ca2_cache_layer_offsets")
+    return t.value, s_.value
+
+
 def ca2_cache_write(handle, k_t, v_t, k_s, v_s, n_frames: int, stream=None) -> None:
     _check(load_library().ca2_cache_write(handle, _ptr_array(k_t), _ptr_array(v_t), _ptr_array(k_s),
                                           _ptr_array(v_s), int(n_frames), _stream(stream)),
@@ -228,7 +252,7 @@ def ca2_cache_state(handle) -> Tuple[int, int, int, int]:
 
 
 def ca2_device_status() -> int:
-    """Returns the status code (0 or CA2_ERR_TIMEOUT / CA2_ERR_CUDA) without raising."""
+    """Returns the status code (0, CA2_ERR_TIMEOUT, CA2_ERR_RANGE or CA2_ERR_CUDA) without raising."""
     return int(load_library().ca2_device_status())
 
 
@@ -244,24 +268,34 @@ def ca2_last_error_string() -> str:
     return load_library().ca2_last_error_string().decode()
 
 
+def _numel(shape) -> int:
+    n = 1
+    for d in shape:
+        n *= int(d)
+    return n
+
+
 # ---- convenience owner ------------------------------------------------------------------
 class KVCache:
     """Cache buffers allocated with torch on the current CUDA device, plus the handle.
 
     ``ring(layer, kv)`` ([B][HW][H][Pmax][D]) and ``spatial(layer, kv)`` ([P'][B][HW][H][D])
-    are bf16 views of the buffers with the layout documented in include/ca2.h.
+    are bf16 views of the buffers with the layout documented in include/ca2.h, at the
+    offsets the library reports.  ``row_pitch`` (elements, 0 = H*D) is the distance between
+    consecutive rows of the caller's chunk tensors.
     """
 
     def __init__(self, n_layers, batch, hw, heads, head_dim, chunk_len, p_max, p_spatial,
-                 tpe_len=0, device=None):
+                 tpe_len=0, device=None, row_pitch=0):
         import torch
-        self.cfg = ca2_config(n_layers, batch, hw, heads, head_dim, chunk_len, p_max, p_spatial, tpe_len)
-        self.tpe_len = tpe_len if tpe_len > 0 else p_max + chunk_len   # rows of the TPE table
-        tb, sb = ca2_cache_bytes(self.cfg)
+        cfg = ca2_config(n_layers, batch, hw, heads, head_dim, chunk_len, p_max, p_spatial, tpe_len, row_pitch)
+        tb, sb = ca2_cache_bytes(cfg)
         dev = device or torch.device("cuda", torch.cuda.current_device())
         self.tbuf = torch.empty(tb // 2, dtype=torch.bfloat16, device=dev)
         self.sbuf = torch.empty(max(sb // 2, 8), dtype=torch.bfloat16, device=dev)
-        self.handle = ca2_cache_init(self.cfg, self.tbuf, tb, self.sbuf if sb else None, sb)
+        self.handle = ca2_cache_init(cfg, self.tbuf, tb, self.sbuf if sb else None, sb)
+        self.cfg = ca2_cache_config(self.handle)         # defaults resolved by the library
+        self.tpe_len = self.cfg.tpe_len                   # rows of the TPE table
 
     def close(self):
         if self.handle:
@@ -277,15 +311,15 @@ class KVCache:
     def ring(self, layer: int, kv: int):
         """Ring of one layer, token-major and head-major within a token: [B][HW][H][Pmax][D]."""
         c = self.cfg
-        per = c.p_max * c.batch * c.hw * c.heads * c.head_dim
-        off = (layer * 2 + kv) * per
-        return self.tbuf[off:off + per].view(c.batch, c.hw, c.heads, c.p_max, c.head_dim)
+        off = ca2_cache_layer_offsets(self.handle, layer, kv)[0] // 2
+        shape = (c.batch, c.hw, c.heads, c.p_max, c.head_dim)
+        return self.tbuf[off:off + _numel(shape)].view(*shape)
 
     def spatial(self, layer: int, kv: int):
         c = self.cfg
-        per = c.p_spatial * c.batch * c.hw * c.heads * c.head_dim
-        off = (layer * 2 + kv) * per
-        return self.sbuf[off:off + per].view(c.p_spatial, c.batch, c.hw, c.heads, c.head_dim)
+        off = ca2_cache_layer_offsets(self.handle, layer, kv)[1] // 2
+        shape = (c.p_spatial, c.batch, c.hw, c.heads, c.head_dim)
+        return self.sbuf[off:off + _numel(shape)].view(*shape)
 
     def state(self):
         return ca2_cache_state(self.handle)
@@ -295,11 +329,7 @@ class KVCache:
 
     def evict_for(self, n_new: int) -> int:
         """Evict just enough of the oldest frames for n_new more to fit; returns that count."""
-        _, count, _, _ = self.state()
-        e = max(0, count + n_new - self.cfg.p_max)
-        if e:
-            self.evict(e)
-        return e
+        return ca2_cache_evict_for(self.handle, n_new)
 
     def write(self, k_t, v_t, k_s, v_s, n, stream=None):
         ca2_cache_write(self.handle, k_t, v_t, k_s, v_s, n, stream)

@@ -4,6 +4,7 @@
 // state of the temporal KV-cache queue (head / count kept on the host and passed to the
 // kernels by value), the spatial-cache frame count, cyclic TPE indices, tensor-map
 // encoding for the tensor-core kernel, and kernel launches on the caller's stream.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -18,7 +19,7 @@
 
 struct ca2_cache {
     ca2_config cfg;
-    uint8_t *tbuf;      // [N_L][2][B][HW][Pmax][H][D] bf16 (token-major ring)
+    uint8_t *tbuf;      // [N_L][2][B][HW][H][Pmax][D] bf16 (token-major, head-major ring)
     uint8_t *sbuf;      // [N_L][2][P'][B][HW][H][D] bf16
     size_t plane_bytes; // bytes of one frame-plane B*HW*H*D*2
     int head;           // ring slot of the oldest queued frame
@@ -43,6 +44,11 @@ int validate_config(const ca2_config *c)
     // tensor-map extents and 32-bit strides
     const long long hd = (long long)c->heads * c->head_dim;
     if (hd * c->hw * 2 > (1ll << 40) || c->hw > (1 << 30)) return CA2_ERR_SHAPE;
+    // rows of the caller's chunk tensors: 16-byte multiples, at least this cache's heads
+    if (c->row_pitch != 0 && (c->row_pitch < hd || (c->row_pitch % 8) != 0 || c->row_pitch > (1 << 24)))
+        return CA2_ERR_SHAPE;
+    const long long pitch = c->row_pitch ? c->row_pitch : hd;
+    if (pitch * c->hw * c->chunk_len * 2 > (1ll << 40)) return CA2_ERR_SHAPE;
     return CA2_OK;
 }
 
@@ -61,41 +67,46 @@ int cuda_status(cudaError_t e)
     return CA2_ERR_CUDA;
 }
 
+// Multiprocessor count of the current device, read once per device (devices past 63 are
+// queried on every call).
 int sm_count()
 {
-    static int cached_dev = -1, cached = 0;
+    static std::atomic<int> cached[64];   // 0 = not read yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev != cached_dev) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        cached = n;
-        cached_dev = dev;
+    if (dev >= 0 && dev < 64) {
+        const int n = cached[dev].load(std::memory_order_relaxed);
+        if (n > 0) return n;
     }
-    return cached;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
+// The driver's tensor-map encoder, looked up once (thread-safe static initialisation).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
-// View a bf16 tensor [frames][HW][H][D] as 4-D (D, H, HW, frames) and encode a tiled map.
-bool encode_4d(CUtensorMap *m, const void *base, int D, int H, int HW, int frames, int box_d, int box_rows,
-               CUtensorMapSwizzle swz)
+// View a bf16 tensor [frames][HW][H][D] whose token rows are `pitch` elements apart as 4-D
+// (D, H, HW, frames) and encode a tiled map.
+bool encode_4d(CUtensorMap *m, const void *base, int D, int H, int HW, int frames, long long pitch, int box_d,
+               int box_rows, CUtensorMapSwizzle swz)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)HW, (cuuint64_t)frames};
-    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)HW * H * D * 2};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)pitch * 2, (cuuint64_t)HW * pitch * 2};
     cuuint32_t box[4] = {(cuuint32_t)box_d, 1u, (cuuint32_t)box_rows, 1u};
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
@@ -190,6 +201,7 @@ int ca2_cache_init(const ca2_config *cfg, void *temporal_buf, size_t temporal_by
     if (!c) return CA2_ERR_ARG;
     c->cfg = *cfg;
     if (c->cfg.tpe_len == 0) c->cfg.tpe_len = cfg->p_max + cfg->chunk_len;
+    if (c->cfg.row_pitch == 0) c->cfg.row_pitch = cfg->heads * cfg->head_dim;
     c->tbuf = static_cast<uint8_t *>(temporal_buf);
     c->sbuf = static_cast<uint8_t *>(spatial_buf);
     c->plane_bytes = plane_bytes_of(cfg);
@@ -207,12 +219,39 @@ int ca2_cache_destroy(ca2_cache *cache)
     return CA2_OK;
 }
 
+int ca2_cache_config(const ca2_cache *c, ca2_config *out)
+{
+    if (!c || !out) return CA2_ERR_ARG;
+    *out = c->cfg;
+    return CA2_OK;
+}
+
+int ca2_cache_layer_offsets(const ca2_cache *c, int layer, int kv, size_t *temporal_offset, size_t *spatial_offset)
+{
+    if (!c || layer < 0 || layer >= c->cfg.n_layers || (kv != 0 && kv != 1)) return CA2_ERR_ARG;
+    if (temporal_offset) *temporal_offset = (size_t)(layer_ring(c, layer, kv) - c->tbuf);
+    if (spatial_offset)
+        *spatial_offset = ((size_t)layer * 2 + (size_t)kv) * (size_t)c->cfg.p_spatial * c->plane_bytes;
+    return CA2_OK;
+}
+
 int ca2_cache_evict(ca2_cache *c, int n)
 {
     if (!c) return CA2_ERR_ARG;
     if (n < 0 || n > c->count) return CA2_ERR_CAPACITY;
     c->head = (c->head + n) % c->cfg.p_max;
     c->count -= n;
+    return CA2_OK;
+}
+
+int ca2_cache_evict_for(ca2_cache *c, int n_new, int *evicted)
+{
+    if (!c) return CA2_ERR_ARG;
+    if (n_new < 0 || n_new > c->cfg.p_max) return CA2_ERR_SHAPE;
+    const int e = c->count + n_new > c->cfg.p_max ? c->count + n_new - c->cfg.p_max : 0;
+    const int st = ca2_cache_evict(c, e);
+    if (st != CA2_OK) return st;
+    if (evicted) *evicted = e;
     return CA2_OK;
 }
 
@@ -237,7 +276,8 @@ int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t
     std::memset(&p, 0, sizeof(p));
     p.tbuf = reinterpret_cast<uint4 *>(c->tbuf);
     p.sbuf = reinterpret_cast<uint4 *>(c->sbuf);
-    p.row_vec = (long long)g.heads * g.head_dim / 8;   // 16-byte vectors per (video, token, frame) row
+    p.row_vec = (long long)g.heads * g.head_dim / 8;   // 16-byte vectors of this cache's heads per row
+    p.src_row_vec = (long long)g.row_pitch / 8;        // 16-byte vectors from one source row to the next
     p.tokens = (long long)g.batch * g.hw;
     p.head_vec = g.head_dim / 8;                       // 16-byte vectors per head row
     p.heads = g.heads;
@@ -292,7 +332,8 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
 
     // temporal chunk tensors are token-major [B][HW][n][H][D] (C = H*D), read as TMA boxes;
     // the ring [B][HW][H][Pmax][D] is read with bulk copies of one head's consecutive slots
-    const long long C = (long long)g.heads * g.head_dim;
+    const long long C = g.row_pitch;                   // elements from one chunk row to the next
+    p.pitch = g.row_pitch;
     p.rk = layer_ring(c, layer, 0);
     p.rv = layer_ring(c, layer, 1);
     ca2::TemporalMaps m;
@@ -321,14 +362,16 @@ int ca2_spatial_prefix_attn(ca2_cache *c, int layer, const void *q, const void *
     const int frames = g.batch * n;
     ca2::SpatialMaps m;
     const int D = g.head_dim, H = g.heads, HW = g.hw;
-    auto load_map = [&](CUtensorMap *mm, const void *base, int frames_) {
-        return encode_4d(mm, base, D, H, HW, frames_, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+    // the caller's chunk rows are row_pitch apart; the spatial cache's rows are H*D apart
+    auto load_map = [&](CUtensorMap *mm, const void *base, int frames_, long long pitch) {
+        return encode_4d(mm, base, D, H, HW, frames_, pitch, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
     };
-    bool ok = load_map(&m.q, q, frames) && load_map(&m.k, k, frames) && load_map(&m.v, v, frames) &&
-              encode_4d(&m.o, out, D, H, HW, frames, D, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    const long long cp = g.row_pitch, hd = (long long)H * D;
+    bool ok = load_map(&m.q, q, frames, cp) && load_map(&m.k, k, frames, cp) && load_map(&m.v, v, frames, cp) &&
+              encode_4d(&m.o, out, D, H, HW, frames, cp, D, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (ok && n_sp > 0) {
-        ok = load_map(&m.sk, layer_spatial(c, layer, 0), n_sp * g.batch) &&
-             load_map(&m.sv, layer_spatial(c, layer, 1), n_sp * g.batch);
+        ok = load_map(&m.sk, layer_spatial(c, layer, 0), n_sp * g.batch, hd) &&
+             load_map(&m.sv, layer_spatial(c, layer, 1), n_sp * g.batch, hd);
     } else if (ok) {
         m.sk = m.k;   // never read when there is no prefix
         m.sv = m.v;
@@ -363,7 +406,8 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     const void *ptrs[6] = {x_t, w_t, b_t, n_sp > 0 ? x_s : nullptr, n_sp > 0 ? w_s : nullptr, n_sp > 0 ? b_s : nullptr};
     for (const void *q : ptrs)
         if (q && !aligned16(q)) return CA2_ERR_ALIGN;
-    const long long C = (long long)g.heads * g.head_dim;
+    const long long C = (long long)g.heads * g.head_dim;   // output channels of K (and of V)
+    const long long Cin = g.row_pitch;                       // input channels: a whole row
     const long long rows_t = (long long)g.batch * g.hw * n;
     if (rows_t >= (1ll << 31) || C * 2 >= (1ll << 31)) return CA2_ERR_SHAPE;
 
@@ -388,19 +432,19 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     p.tiles_n = (int)((2 * C + ca2::kProjBN - 1) / ca2::kProjBN);
     p.tiles_t = (int)((rows_t + 127) / 128) * p.tiles_n;
     p.tiles_s_frame = (g.hw + 127) / 128;
-    p.k_steps = (int)((C + 63) / 64);
+    p.k_steps = (int)((Cin + 63) / 64);
     const long long tiles_s = (long long)g.batch * n_sp * p.tiles_s_frame * p.tiles_n;
     if (p.tiles_t + tiles_s >= (1ll << 31)) return CA2_ERR_SHAPE;
     p.total_tiles = (int)(p.tiles_t + tiles_s);
 
-    // x_t: [B*HW*n][C]; x_s: (C, HW, B*n frames); W: [2C][C] (output channel rows)
+    // x_t: [B*HW*n][Cin]; x_s: (Cin, HW, B*n frames); W: [2C][Cin] (output channel rows)
     ca2::KvProjMaps m;
     std::memset(&m, 0, sizeof(m));
-    bool ok = encode_rows_3d(&m.xt, x_t, C, rows_t, 1, C, rows_t * C, 128) &&
-              encode_rows_3d(&m.wt, w_t, C, 2 * C, 1, C, 2 * C * C, ca2::kProjBN);
+    bool ok = encode_rows_3d(&m.xt, x_t, Cin, rows_t, 1, Cin, rows_t * Cin, 128) &&
+              encode_rows_3d(&m.wt, w_t, Cin, 2 * C, 1, Cin, 2 * C * Cin, ca2::kProjBN);
     if (ok && n_sp > 0)
-        ok = encode_rows_3d(&m.xs, x_s, C, g.hw, (long long)g.batch * n, C, (long long)g.hw * C, 128) &&
-             encode_rows_3d(&m.ws, w_s, C, 2 * C, 1, C, 2 * C * C, ca2::kProjBN);
+        ok = encode_rows_3d(&m.xs, x_s, Cin, g.hw, (long long)g.batch * n, Cin, (long long)g.hw * Cin, 128) &&
+             encode_rows_3d(&m.ws, w_s, Cin, 2 * C, 1, Cin, 2 * C * Cin, ca2::kProjBN);
     else
         m.xs = m.xt, m.ws = m.wt;    // no spatial tile reads them
     if (!ok) {
@@ -441,8 +485,10 @@ int ca2_tpe_add(const ca2_cache *c, long long first_global_frame, int offset, co
     p.table = static_cast<const uint4 *>(table);
     p.rows = (long long)g.batch * g.hw * n;
     p.row_vec = g.heads * g.head_dim / 8;
+    p.pitch_vec = g.row_pitch / 8;
     p.n = n;
-    if (p.rows * p.row_vec >= (1ll << 31)) return CA2_ERR_SHAPE;   // the kernel indexes in 32 bits
+    // the kernel indexes in 32 bits
+    if (p.rows * p.pitch_vec >= (1ll << 31) || (long long)n_tpe * p.pitch_vec >= (1ll << 31)) return CA2_ERR_SHAPE;
     for (int i = 0; i < ca2::kMaxChunk; ++i)
         p.tpe_row[i] = i < n ? (int)(((long long)offset + first_global_frame + i) % n_tpe) : 0;
     return cuda_status(ca2::launch_tpe_add(p, static_cast<cudaStream_t>(stream)));
@@ -473,7 +519,8 @@ int ca2_device_status(void)
     if (cudaDeviceSynchronize() != cudaSuccess) return CA2_ERR_CUDA;
     int s = 0;
     if (ca2::read_and_clear_status(&s) != 0) return CA2_ERR_CUDA;
-    return s == 0 ? CA2_OK : CA2_ERR_TIMEOUT;
+    if (s == 0) return CA2_OK;
+    return s >= ca2::kStatusRangeCode ? CA2_ERR_RANGE : CA2_ERR_TIMEOUT;
 }
 
 int ca2_selftest_timeout(int wait_us, void *stream)
@@ -495,6 +542,7 @@ const char *ca2_status_string(int s)
     case CA2_ERR_ALIGN: return "pointer not 16-byte aligned";
     case CA2_ERR_CUDA: return "CUDA runtime error";
     case CA2_ERR_TIMEOUT: return "device wait timed out";
+    case CA2_ERR_RANGE: return "input value outside the supported range";
     default: return "unknown status";
     }
 }

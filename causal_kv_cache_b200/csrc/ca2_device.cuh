@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace ca2 {
 
@@ -26,6 +27,15 @@ __device__ __forceinline__ unsigned long long global_ns()
 __device__ __forceinline__ void record_timeout(int site)
 {
     atomicCAS(&g_status, 0, site);
+}
+
+// Status codes of kStatusRange and above mean an input outside the supported range (not a
+// timeout); the first record wins, as for timeouts.  (The same value as kStatusRangeCode,
+// which the host side reads.)
+constexpr int kStatusRange = 1000;
+__device__ __forceinline__ void record_status(int code)
+{
+    atomicCAS(&g_status, 0, code);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -215,6 +225,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
 // The two bf16 halves of a packed word, widened exactly to fp32.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Per-halfword maximum of the magnitude bits of four words of bf16 pairs (the sign bit is
+// cleared before the max, so a negative value never hides a larger magnitude).
+__device__ __forceinline__ uint32_t abs_max4(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __vmaxu2(__vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu), __vmaxu2(c & 0x7FFF7FFFu, d & 0x7FFF7FFFu));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);              // .x = lo (low half), .y = hi
+    return *reinterpret_cast<uint32_t *>(&v);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {

@@ -1,6 +1,7 @@
 // ca2_kernels.h -- launch interface between the C-ABI layer (ca2_api.cu) and the kernels.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -29,6 +30,21 @@ inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 bloc
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Raise a kernel's dynamic shared-memory limit on the current device, once per device.
+// `configured` is the launch site's own record (bit d = done on device d); concurrent callers
+// may both set the attribute, which is harmless.  Devices past 63 set it on every call.
+inline cudaError_t ensure_smem_attr(std::atomic<uint64_t> &configured, const void *func, int bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (configured.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) configured.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
 // ---- causal temporal attention ---------------------------------------------------------
 // heads per work item = consumer warps per CTA.  Two heads and four stages make CTAs of
 // ~42 KB of shared memory at D = 72, five per SM: more independent consumer warps per SM
@@ -41,6 +57,7 @@ struct TemporalParams {
     __nv_bfloat16 *out;                 // [B][HW][n][H][D]
     const uint8_t *rk, *rv;             // this layer's K and V rings [B][HW][H][Pmax][D]
     int B, HW, H, D;
+    long long pitch;  // elements from one row of a chunk tensor to the next (>= H * D)
     int n;          // chunk frames in this call (queries per token-head)
     int Pk;         // queued frames
     int head;       // ring slot of the oldest queued frame
@@ -73,7 +90,8 @@ struct CacheWriteParams {
     CacheWriteLayer layer[kMaxLayersPerWrite];
     uint4 *tbuf;            // temporal cache base [N_L][2][B][HW][H][Pmax][D] (token-major, head-major ring)
     uint4 *sbuf;            // spatial cache base  [N_L][2][P'][B][HW][C]
-    long long row_vec;      // 16-byte vectors per row of C = H*D elements
+    long long row_vec;      // 16-byte vectors of this cache's C = H*D channels in a row
+    long long src_row_vec;  // 16-byte vectors from one source row to the next (row pitch / 8)
     int head_vec;           // 16-byte vectors per head row of D elements
     int heads;
     long long tokens;       // B * HW
@@ -113,7 +131,8 @@ struct TpeAddParams {
     uint4 *out;             // same layout; may equal x
     const uint4 *table;     // [N_tpe][C]
     long long rows;         // B * HW * n
-    int row_vec;            // 16-byte vectors per row of C = H*D elements
+    int row_vec;            // 16-byte vectors of the C = H*D channels added per row
+    int pitch_vec;          // 16-byte vectors from one row of x, out or table to the next
     int n;                  // chunk frames
     int tpe_row[kMaxChunk]; // table row of each chunk frame
 };
@@ -154,6 +173,11 @@ struct KvProjMaps {
 };
 
 cudaError_t launch_kv_proj(const KvProjMaps &maps, const KvProjParams &p, int grid, cudaStream_t stream);
+
+// ---- device status word -------------------------------------------------------------------
+// 0 = fine; codes below kStatusRangeCode name the bounded wait that gave up, codes from it on
+// an input value outside the supported range (device code records them with record_status).
+constexpr int kStatusRangeCode = 1000;
 
 // ---- bounded-wait self test ---------------------------------------------------------------
 cudaError_t launch_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);

@@ -33,6 +33,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 // blockIdx.y = (layer, tensor): tensor 0/1 = temporal K/V, 2/3 = spatial K/V.
 //   temporal: chunk [B][HW][n][H][D] -> ring [B][HW][H][Pmax][D]; (token, j, h) -> slot (slot0 + j) mod Pmax
 //   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
+//             (K copied, V converted to fp16)
+// (source rows are src_row_vec 16-byte vectors apart, of which the first row_vec are copied)
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
     const int li = blockIdx.y >> 2;
@@ -69,18 +71,32 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
                 if (slot >= p.p_max) slot -= p.p_max;
                 const int h = (int)(off / p.head_vec);
                 const long long dv = off - (long long)h * p.head_vec;
-                so[i] = e;
+                so[i] = row * p.src_row_vec + off;
                 dof[i] = ((tok * p.heads + h) * p.p_max + slot) * p.head_vec + dv;
             } else {
                 // row = jsp * tokens + (b * HW + s); source frame n - n_sp + jsp of video b
                 const long long jsp = row / p.tokens;
                 const long long bt = row - jsp * p.tokens;
                 const long long b = bt / p.hw, sidx = bt - b * p.hw;
-                so[i] = ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * rv + off;
+                so[i] = ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * p.src_row_vec + off;
                 dof[i] = e;
             }
             v[i] = ld_stream(src + so[i]);
         }
+    }
+    if (tensor == 3) {
+        // the spatial cache keeps V in fp16, the operand type of the spatial attention's P V
+        // product: the exact value of each bf16 element within the fp16 range; elements
+        // beyond it (|v| >= 65536, inf, NaN) are recorded as a range error
+        uint32_t vmax = 0;
+#pragma unroll
+        for (int i = 0; i < kVecPerThread; ++i) {
+            if (dof[i] < 0) continue;
+            vmax = __vmaxu2(vmax, abs_max4(v[i].x, v[i].y, v[i].z, v[i].w));
+            v[i] = make_uint4(pack_f16x2(bf16_lo(v[i].x), bf16_hi(v[i].x)), pack_f16x2(bf16_lo(v[i].y), bf16_hi(v[i].y)),
+                              pack_f16x2(bf16_lo(v[i].z), bf16_hi(v[i].z)), pack_f16x2(bf16_lo(v[i].w), bf16_hi(v[i].w)));
+        }
+        if ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u) record_status(kStatusRange);
     }
 #pragma unroll
     for (int i = 0; i < kVecPerThread; ++i)

@@ -28,6 +28,7 @@
 // zero-filled by the TMA unit; the epilogue skips rows and channels that do not exist.
 // Every mbarrier wait is bounded; a timeout is recorded in the library status word and all
 // roles wind down (issued copies land, issued MMAs complete, TMEM is freed).
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
         const int quarter = warp & 3;                     // TMEM lanes 32 * quarter ..
         const int r = quarter * 32 + lane;                // row of the tile = TMEM lane
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        uint32_t vmax = 0;                                // per-half max of the spatial V bits stored
         int i = 0;
         for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++i) {
             const int acc = i & 1;
@@ -259,6 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
                     w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + b8[2], __uint_as_float(v[8 * q + 3]) + b8[3]);
                     w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) + b8[4], __uint_as_float(v[8 * q + 5]) + b8[5]);
                     w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) + b8[6], __uint_as_float(v[8 * q + 7]) + b8[7]);
+                    if (d.spatial && kv) {
+                        // the spatial cache keeps V in fp16: the exact value of the bf16 result
+                        // within the fp16 range, larger values recorded as a range error
+                        vmax = __vmaxu2(vmax, abs_max4(w.x, w.y, w.z, w.w));
+                        w = make_uint4(pack_f16x2(bf16_lo(w.x), bf16_hi(w.x)), pack_f16x2(bf16_lo(w.y), bf16_hi(w.y)),
+                                       pack_f16x2(bf16_lo(w.z), bf16_hi(w.z)), pack_f16x2(bf16_lo(w.w), bf16_hi(w.w)));
+                    }
                     __nv_bfloat16 *dst = (kv ? dst_v : dst_k) + base + (long long)h * head_stride + dd;
                     *reinterpret_cast<uint4 *>(dst) = w;
                 }
@@ -268,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty(acc));
         }
+        if ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u) record_status(kStatusRange);
     }
     tc_fence_before();
     __syncthreads();
@@ -279,14 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
 
 cudaError_t launch_kv_proj(const KvProjMaps &m, const KvProjParams &p, int grid, cudaStream_t stream)
 {
-    static int configured_for = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_for != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k_kv_proj, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured_for = dev;
-    }
+    static std::atomic<uint64_t> configured{0};
+    const cudaError_t e = ensure_smem_attr(configured, reinterpret_cast<const void *>(&k_kv_proj), (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
     if (grid <= 0) return cudaSuccess;
     return launch_chained(k_kv_proj, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, m, p);
 }

@@ -12,10 +12,12 @@
 //                independent rings (K is released as soon as both QK^T products have read
 //                it, V after both P V products).  An operand tile is ceil(D/32) boxes of 32
 //                head-dims x 128 tokens (64-byte rows, 64-byte swizzle); columns past D
-//                (72 -> 96) and rows past HW are zero-filled by the TMA unit.  When D is
-//                not a multiple of 32, padding column D of each landed V tile is set to 1.0
-//                (by warp 3), so the P V product also accumulates the row sum of the
-//                probabilities into O[:, D].
+//                (72 -> 96) and rows past HW are zero-filled by the TMA unit.  Warp 3
+//                converts each landed V tile in place to fp16, and when D is not a multiple
+//                of 32 sets padding column D to 1.0, so the P V product also accumulates the
+//                row sum of the probabilities into O[:, D].  P V runs in fp16 x fp16: the
+//                probabilities carry 11 significant bits, where bf16 P (8 bits) put an error
+//                of the order of the output's own bf16 rounding into every output.
 //   warps 1, 2   MMA issuers of tile A and tile B (the whole warp runs the loop, one
 //                elected lane issues; warp 1 owns the 512 TMEM columns).  A divergent
 //                single thread issued about one tcgen05.mma per ~100 cycles, the whole warp
@@ -23,7 +25,7 @@
 //                tile's next QK^T is issued as soon as its softmax warps have read the
 //                current scores, and its P V product chunk by chunk as the probabilities
 //                land, so the tensor core works while the exponentials run.
-//   warp 3       prepares each landed V tile (the padding column of ones, below).
+//   warp 3       prepares each landed V tile (fp16 conversion and the padding column, below).
 //   warps 4-11   softmax: 4 warps per tile, one thread per query row (its TMEM lane; warp
 //                % 4 selects the lane quarter) holding all 128 scores of a block in
 //                registers, so the row max needs no exchange.  The exponential unit
@@ -40,9 +42,11 @@
 //
 // Every mbarrier wait is bounded; a timeout is recorded in the library status word and
 // all roles wind down through the common exit, which frees TMEM.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "ca2_device.cuh"
 #include "ca2_kernels.h"
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         const int X = warp - 1;
         const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
         constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16(kRows, DP, false, true);
+        constexpr uint32_t idesc_pv = idesc_f16(kRows, DP, false, true);    // P and V both fp16
         // Descriptors are built once; a k-step only adds its byte offset / 16 to the
         // start-address field (addresses stay below 256 KB, so no carry leaves it).
         // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
@@ -427,30 +431,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         __syncwarp();
     } else if (warp == 3) {
         // ------------------------------- V preparation (one warp) ---------------------
-        // When D is not a multiple of 32, column D of each landed V tile := 1.0 (bf16
-        // 0x3F80) at its swizzled address (64-byte rows, 16-byte chunk index ^= (row >> 1)
-        // & 3), four rows per lane; then the tile is ready for the P V products
+        // The spatial cache holds V in fp16 already (written so once per AR step); a V tile
+        // of the frame's own K/V (bf16, from the caller) is converted in place to fp16 (exact
+        // for |v| in [2^-14, 65504]; smaller values become fp16 subnormals, within 2^-25 of
+        // v): the 16-byte pieces holding columns < D, four rows per lane, whatever their
+        // swizzled position (64-byte rows, 16-byte piece index ^= (row >> 1) & 3).  Values
+        // beyond the fp16 range (|v| >= 65536 in bf16, inf, NaN) are recorded in the library
+        // status word (ca2_device_status reports CA2_ERR_RANGE).  When D is not a multiple of
+        // 32, column D := 1.0 (fp16 0x3C00), so the P V product also accumulates the row sum.
+        const int D = p.D;
+        const int pieces = D >> 3;                        // 16-byte pieces of a row holding columns < D
+        uint32_t vmax = 0;                                // per-half max of |v| bits seen
         auto prep = [&](int jv) -> bool {
             const int s = jv % NS;
             if (!warp_wait(bar(B_VFULL + s), (jv / NS) & 1, 203, abort_flag)) return false;
+            const uint32_t vt = sb + L.v0 + s * TB;
+            // block jv comes from the own frame when its source index is 0 (see kv_src)
+            const bool own = p.n_src == 1 || (jv / p.nkb + 1) % p.n_src == 0;
+            for (int r = lane; own && r < kKeys; r += 32) {
+                const uint32_t rbase = vt + (uint32_t)r * 64u;
+                const uint32_t swz = (uint32_t)((r >> 1) & 3);
+                for (int q = 0; q < pieces; ++q) {
+                    const uint32_t a = rbase + (uint32_t)(q >> 2) * 8192u + ((((uint32_t)q & 3u) ^ swz) << 4);
+                    uint32_t w[4];
+                    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
+                    vmax = __vmaxu2(vmax, abs_max4(w[0], w[1], w[2], w[3]));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) w[i] = pack_f16x2(bf16_lo(w[i]), bf16_hi(w[i]));
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+            }
             if (ones_col) {
-                const uint32_t vt = sb + L.v0 + s * TB;
-                const int D = p.D;
                 const int c = (D & 31) >> 3;
                 const uint32_t base = vt + (uint32_t)(D >> 5) * 8192u + (uint32_t)((D & 7) * 2);
 #pragma unroll
                 for (int r = lane; r < kKeys; r += 32)
                     asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) << 4)),
-                                 "h"((unsigned short)0x3F80)
+                                 "h"((unsigned short)0x3C00)
                                  : "memory");
-                fence_proxy_async_smem();
             }
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_VREADY + s));
             return true;
         };
         for (int j = 0; j < NB; ++j)
             if (!prep(j)) break;
+        if ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u) record_status(kStatusRange);
     } else if (warp >= kSoftmaxWarp0) {
         // ------------------------------- softmax / epilogue ---------------------------
         // 8 warps: tile X = (warp - 4) / 4, lane quarter = warp % 4, one thread per query
@@ -539,8 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 float ls = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    w[i] = pack_bf16x2(e[2 * i], e[2 * i + 1]);
-                    if (!ones_col) ls += bf16_lo(w[i]) + bf16_hi(w[i]);
+                    w[i] = pack_f16x2(e[2 * i], e[2 * i + 1]);
+                    if (!ones_col) ls += e[2 * i] + e[2 * i + 1];
                 }
                 l_sum += ls;
                 if constexpr (kPSmem) {
@@ -649,15 +677,10 @@ template <int NKD>
 static cudaError_t launch_nkd(const SpatialMaps &m, const SpatialParams &p, cudaStream_t stream)
 {
     constexpr uint32_t smem = spatial_layout(NKD).total < kMinSmem ? kMinSmem : spatial_layout(NKD).total;
-    static int configured_for = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_for != dev) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_spatial_prefix<NKD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured_for = dev;
-    }
+    static std::atomic<uint64_t> configured{0};
+    const cudaError_t e =
+        ensure_smem_attr(configured, reinterpret_cast<const void *>(&k_spatial_prefix<NKD>), (int)smem);
+    if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(p.B * p.n * p.H * p.q_pairs);
     return launch_chained(k_spatial_prefix<NKD>, dim3(grid), dim3(kThreads), smem, stream, m, p);
 }

@@ -32,16 +32,19 @@
 //     products use mma.sync on registers: S^T = K Q^T (keys on M, the 8 queries on N),
 //     then O^T += V^T P^T.  Each lane owns the same two query columns in both
 //     accumulators, so the online-softmax rescale is lane-local; movmatrix turns P^T
-//     into the B operand and O^T back into rows for the stores.  The reference max of the
-//     exponentials moves only when a score exceeds it by more than 2^8 (one warp vote per
-//     stage; the max reduction and the rescale run only then), which leaves each softmax
-//     row unchanged after normalisation.
+//     into the B operand and O^T back into rows for the stores.  P enters the product as
+//     two bf16 parts (P rounded, then the remainder rounded), so the probabilities carry
+//     16 significant bits rather than 8.  The reference max of the exponentials moves
+//     only when a score exceeds it by more than 2^8 (one warp vote per stage; the max
+//     reduction and the rescale run only then), which leaves each softmax row unchanged
+//     after normalisation.
 //   * Ring rows that hold no queued frame are masked, and their V rows are zero, so stale
 //     bits (of the caller's buffer or of an earlier stage) never reach the accumulator.
 //     The producer zeroes the V rows past Pmax, which the ring copy does not write, before
 //     it arms the stage (off the consumers' path), so the consumers write shared memory
 //     (and fence it against the next copy into the stage) only for slots inside Pmax that
 //     hold no queued frame, which happens only while the queue fills.
+#include <atomic>
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -438,13 +441,22 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         acc[t][3] *= al1;
                     }
                 }
-                // probabilities rounded to bf16; the normaliser sums the rounded values
-                const uint32_t x0 = pack_bf16x2(ex2(sc[0] - m_run[0]), ex2(sc[1] - m_run[1]));
-                const uint32_t x1 = pack_bf16x2(ex2(sc[2] - m_run[0]), ex2(sc[3] - m_run[1]));
-                l_part[0] += bf16_lo(x0) + bf16_lo(x1);
-                l_part[1] += bf16_hi(x0) + bf16_hi(x1);
+                // probabilities as a bf16 pair hi + lo (hi = P rounded to bf16, lo = the rest
+                // rounded to bf16: 16 significant bits between them), each multiplied by V^T on
+                // the tensor core; a single bf16 P would carry up to 2^-9 relative error into
+                // every output, the same order as the output's own rounding
+                const float e0 = ex2(sc[0] - m_run[0]), e1 = ex2(sc[1] - m_run[1]);
+                const float e2 = ex2(sc[2] - m_run[0]), e3 = ex2(sc[3] - m_run[1]);
+                const uint32_t x0 = pack_bf16x2(e0, e1);
+                const uint32_t x1 = pack_bf16x2(e2, e3);
+                const uint32_t r0 = pack_bf16x2(e0 - bf16_lo(x0), e1 - bf16_hi(x0));
+                const uint32_t r1 = pack_bf16x2(e2 - bf16_lo(x1), e3 - bf16_hi(x1));
+                l_part[0] += e0 + e2;
+                l_part[1] += e1 + e3;
                 const uint32_t pb0 = movm_t(x0);
                 const uint32_t pb1 = movm_t(x1);
+                const uint32_t pl0 = movm_t(r0);
+                const uint32_t pl1 = movm_t(r1);
                 // O^T += V^T P^T, 16 head dims per m-tile
 #pragma unroll
                 for (int t = 0; t < DT; ++t) {
@@ -454,11 +466,13 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         ldsm_x4_t(vbase + (uint32_t)((lane & 7) + 8 * (j >> 1)) * row + (uint32_t)(16 * t + 8 * (j & 1)) * 2u,
                                   a0, a1, a2, a3);
                         mma16816(acc[t], a0, a1, a2, a3, pb0, pb1);
+                        mma16816(acc[t], a0, a1, a2, a3, pl0, pl1);
                     } else {
                         uint32_t a0, a2;
                         ldsm_x2_t(vbase + (uint32_t)((lane & 7) + 8 * ((lane >> 3) & 1)) * row + (uint32_t)(16 * t) * 2u,
                                   a0, a2);
                         mma16816(acc[t], a0, 0u, a2, 0u, pb0, pb1);
+                        mma16816(acc[t], a0, 0u, a2, 0u, pl0, pl1);
                     }
                 }
                 __syncwarp();
@@ -476,7 +490,7 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
             }
             const float i0 = 1.f / l0, i1 = 1.f / l1;
             const int qrow = lane >> 2;
-            __nv_bfloat16 *orow = p.out + (((long long)b * p.HW + s) * p.n + qrow) * (long long)(p.H * D) +
+            __nv_bfloat16 *orow = p.out + (((long long)b * p.HW + s) * p.n + qrow) * p.pitch +
                                   (long long)(hg * G + w) * D + 2 * (lane & 3);
 #pragma unroll
             for (int t = 0; t < DT; ++t) {
@@ -498,15 +512,10 @@ template <int DT>
 static cudaError_t launch_dt(const TemporalMaps &m, const TemporalParams &p, int grid, cudaStream_t stream)
 {
     const uint32_t smem = make_layout(p.G, p.D).total;
-    static int configured_for = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_for != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k_temporal_causal<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)make_layout(kMaxTemporalGroup, 16 * DT).total);
-        if (e != cudaSuccess) return e;
-        configured_for = dev;
-    }
+    static std::atomic<uint64_t> configured{0};
+    const cudaError_t e = ensure_smem_attr(configured, reinterpret_cast<const void *>(&k_temporal_causal<DT>),
+                                           (int)make_layout(kMaxTemporalGroup, 16 * DT).total);
+    if (e != cudaSuccess) return e;
     return launch_chained(k_temporal_causal<DT>, dim3(grid), dim3(32 * (p.G + 1)), smem, stream, m.q, m.k, m.v, p);
 }
 

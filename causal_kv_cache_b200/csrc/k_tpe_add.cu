@@ -36,11 +36,12 @@ __global__ void __launch_bounds__(kThreads) k_tpe_add(const TpeAddParams p)
     // the chunk is produced by the previous kernel on the stream
     wait_previous_kernel();
     allow_next_kernel();
-    // 32-bit index arithmetic: the host guarantees rows * row_vec < 2^31
+    // 32-bit index arithmetic: the host guarantees rows * pitch_vec < 2^31
     const uint32_t total = (uint32_t)(p.rows * (long long)p.row_vec);
-    const uint32_t rv = (uint32_t)p.row_vec, n = (uint32_t)p.n;
+    const uint32_t rv = (uint32_t)p.row_vec, pv = (uint32_t)p.pitch_vec, n = (uint32_t)p.n;
     const uint32_t base = blockIdx.x * (uint32_t)(kThreads * kVecPerThread) + threadIdx.x;
     uint4 xv[kVecPerThread], tv[kVecPerThread];
+    uint32_t xi[kVecPerThread];
 #pragma unroll
     for (int i = 0; i < kVecPerThread; ++i) {
         const uint32_t e = base + (uint32_t)(i * kThreads);
@@ -48,14 +49,15 @@ __global__ void __launch_bounds__(kThreads) k_tpe_add(const TpeAddParams p)
             const uint32_t row = e / rv;                    // (video, token, frame) row
             const uint32_t v = e - row * rv;                // 16-byte vector within the row
             const uint32_t f = row % n;                     // chunk frame (token-major rows)
-            xv[i] = p.x[e];
-            tv[i] = p.table[(uint32_t)p.tpe_row[f] * rv + v];
+            xi[i] = row * pv + v;
+            xv[i] = p.x[xi[i]];
+            tv[i] = p.table[(uint32_t)p.tpe_row[f] * pv + v];
         }
     }
 #pragma unroll
     for (int i = 0; i < kVecPerThread; ++i) {
         const uint32_t e = base + (uint32_t)(i * kThreads);
-        if (e < total) p.out[e] = add8(xv[i], tv[i]);
+        if (e < total) p.out[xi[i]] = add8(xv[i], tv[i]);
     }
 }
 

@@ -14,7 +14,11 @@
  *     of the chunk, spatial token, head, head dim -- the (B*T) x S x C view a spatial block
  *     works in.  Temporal chunk tensors (q, k, v, out of the temporal call and the k_t, v_t
  *     given to the cache write) are token-major [B][HW][n][H][D] -- the (B*S) x T x C view a
- *     temporal block works in.  All device pointers must be 16-byte aligned.
+ *     temporal block works in.  A row (one token of one frame) holds the H*D elements of
+ *     this cache's heads; consecutive rows are cfg.row_pitch elements apart (default H*D),
+ *     so a caller whose activations carry more heads (a rank owning heads [h0, h0+H) of a
+ *     wider model) passes pointers to element h0*D of the first row and the full width as
+ *     row_pitch.  All device pointers must be 16-byte aligned.
  *   - The caller owns all device memory (allocate it however you like, e.g. torch).
  *     The library stores the two cache pointers given to ca2_cache_init and never
  *     frees or reallocates them.
@@ -31,7 +35,9 @@
  *   temporal: [N_L][2][B][HW][H][Pmax][D]   (index 0 = K ring, 1 = V ring; token-major and
  *                                            head-major within a token: one head's Pmax
  *                                            slots are contiguous)
- *   spatial : [N_L][2][P'][B][HW][H][D]
+ *   spatial : [N_L][2][P'][B][HW][H][D]     (K in bf16; V in fp16, the operand type of the
+ *                                            spatial attention's P V product: each bf16 value
+ *                                            converted exactly, |v| <= 65504)
  * The i-th oldest queued frame (i = 0 .. count-1) is in ring slot (head + i) mod Pmax;
  * spatial slot j (j < sp_count) holds the j-th of the last sp_count frames written,
  * oldest first.  Slots that hold no queued frame may contain anything: they are masked,
@@ -40,7 +46,7 @@
  * Required order within one AR step:
  *   T x { for each layer: ca2_spatial_prefix_attn(use_prefix=1), ca2_temporal_attn }
  *   cache-writing pass: for each layer: ca2_spatial_prefix_attn(use_prefix=0), ca2_temporal_attn
- *   ca2_cache_evict(max(0, count + n - Pmax))   then   ca2_cache_write(n)
+ *   ca2_cache_evict_for(n) (evicts max(0, count + n - Pmax) frames)   then   ca2_cache_write(n)
  * The pass's attention reads the queue before eviction overwrites its oldest slots;
  * stream order keeps that true on the device.
  */
@@ -65,6 +71,8 @@ typedef struct {
     int p_max;      /* l <= Pmax <= 512: capacity of the temporal queue, in frames         */
     int p_spatial;  /* P': 0 <= P' <= l prefix frames kept for spatial attention           */
     int tpe_len;    /* N_tpe >= 1: temporal positional table length; 0 selects Pmax + l     */
+    int row_pitch;  /* elements from one row of a chunk tensor to the next: 0 selects H*D,
+                       else a multiple of 8, >= H*D (the activations' full width)          */
 } ca2_config;
 
 typedef enum {
@@ -74,7 +82,9 @@ typedef enum {
     CA2_ERR_CAPACITY = -3,  /* write would overflow the queue, or a buffer is too small   */
     CA2_ERR_ALIGN = -4,     /* a pointer is not 16-byte aligned                           */
     CA2_ERR_CUDA = -5,      /* a CUDA runtime call or kernel launch failed                */
-    CA2_ERR_TIMEOUT = -6    /* a kernel's bounded wait gave up (see ca2_device_status)     */
+    CA2_ERR_TIMEOUT = -6,   /* a kernel's bounded wait gave up (see ca2_device_status)     */
+    CA2_ERR_RANGE = -7      /* a device input outside the supported range (see
+                               ca2_device_status): spatial attention takes |V| <= 65504    */
 } ca2_status;
 
 /* Sizes in bytes of the temporal and spatial cache buffers for a configuration:
@@ -93,19 +103,40 @@ int ca2_cache_init(const ca2_config *cfg, void *temporal_buf, size_t temporal_by
 /* Release the handle (not the caller's buffers).  NULL is accepted. */
 int ca2_cache_destroy(ca2_cache *cache);
 
+/* The handle's configuration with the defaults resolved (tpe_len = Pmax + l and row_pitch =
+ * H*D when given as 0).  Host-only. */
+int ca2_cache_config(const ca2_cache *cache, ca2_config *out);
+
+/* Byte offsets, within the temporal and the spatial cache buffer, of layer `layer`'s K
+ * (kv = 0) or V (kv = 1) ring [B][HW][H][Pmax][D] and spatial cache [P'][B][HW][H][D], for
+ * callers that inspect or fill them.  Either out pointer may be NULL.  Host-only. */
+int ca2_cache_layer_offsets(const ca2_cache *cache, int layer, int kv, size_t *temporal_offset,
+                            size_t *spatial_offset);
+
 /* Dequeue the n oldest queued frames (papernotes page, 关键设计 4: once the queue reaches
  * Pmax the earliest cache entries leave it).  Host-only: head = (head + n) mod Pmax,
  * count -= n.  0 <= n <= count, else CA2_ERR_CAPACITY. */
 int ca2_cache_evict(ca2_cache *cache, int n_frames);
 
+/* Make room for n_new frames (papernotes page, 关键设计 4: once the queue reaches Pmax its
+ * earliest entries leave it): evict exactly e = max(0, count + n_new - Pmax) oldest frames, as
+ * ca2_cache_evict(e), and store e in *evicted (may be NULL).  Host-only.
+ * 0 <= n_new <= Pmax, else CA2_ERR_SHAPE (nothing evicted). */
+int ca2_cache_evict_for(ca2_cache *cache, int n_new, int *evicted);
+
 /* Cache-writing stage (papernotes page, 整体框架 and 关键设计 4-5).  For every layer L:
  * frames j = 0..n-1 of k_t[L], v_t[L] are copied into ring slots
  * (head + count + j) mod Pmax; then the spatial cache of layer L is overwritten with the
  * last min(P', n) frames of k_s[L], v_s[L].  count += n.  One kernel launch for all
- * layers; a bit-exact copy.  k_t[L], v_t[L] are token-major [B][HW][n][H][D]; k_s[L],
+ * layers; a bit-exact copy, except that the spatial V is stored as fp16 (the same values;
+ * |v| >= 65536, inf or NaN there is recorded as CA2_ERR_RANGE, read by ca2_device_status).
+ * k_t[L], v_t[L] are token-major [B][HW][n][H][D]; k_s[L],
  * v_s[L] are frame-major [B][n][HW][H][D].  k_t, v_t, k_s, v_s are HOST arrays of N_L
- * device pointers (k_s, v_s may be NULL when P' = 0).  1 <= n <= l; count + n > Pmax is
- * CA2_ERR_CAPACITY (evict first). */
+ * device pointers (k_s, v_s may be NULL when P' = 0); their rows are row_pitch elements
+ * apart.  1 <= n <= l; count + n > Pmax is CA2_ERR_CAPACITY (evict first).  Every argument
+ * of every layer is validated before the first launch; the write is one launch per 64
+ * layers, and if a later launch fails (CA2_ERR_CUDA) the queue state does not advance and
+ * the cache contents of the layers already written are undefined until the next write. */
 int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const *v_t,
                     const void *const *k_s, const void *const *v_s, int n_frames, void *stream);
 
@@ -116,11 +147,13 @@ int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const 
  *             frame f go to ring slot (head + count + f) mod Pmax of layer `layer`;
  *   spatial : [K | V] = x_s w_s^T + b_s for the chunk's last n_sp = min(P', n) frames of
  *             x_s; frame f goes to spatial-cache frame f - (n - n_sp).
- * x_t: token-major [B][HW][n][C] (C = H*D); x_s: frame-major [B][n][HW][C]; w_t, w_s:
- * [2C][C] row-major, row o = output channel o (K channels 0..C-1 as (head, dim), then V);
+ * x_t: token-major [B][HW][n][Cin]; x_s: frame-major [B][n][HW][Cin], where Cin = row_pitch
+ * (every element of a row is an input channel; Cin = C = H*D by default); w_t, w_s:
+ * [2C][Cin] row-major, row o = output channel o (K channels 0..C-1 as (head, dim), then V);
  * b_t, b_s: [2C] or NULL for no bias.  All bf16, device memory, 16-byte aligned.  fp32
  * accumulation on the tensor cores, then the bias, then one rounding to bf16 (nearest,
- * ties to even).  x_s, w_s, b_s are not read when n_sp = 0 (may be NULL).
+ * ties to even); the spatial V is stored as the fp16 of that bf16 value (see the cache
+ * layout above).  x_s, w_s, b_s are not read when n_sp = 0 (may be NULL).
  * The queue does not advance: after this call for every layer, call ca2_cache_commit(n)
  * (evict first, as for ca2_cache_write).  1 <= n <= chunk_len and count + n <= Pmax, else
  * CA2_ERR_SHAPE / CA2_ERR_CAPACITY.  Asynchronous on `stream`. */
@@ -153,7 +186,10 @@ int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k,
  * use_prefix = 0 (clean prefix frames, the cache-writing pass): keys/values are frame f's
  *   own tokens repeated P'+1 times; repetition leaves softmax attention unchanged, so
  *   the kernel reads them once.
- * q, k, v, out: frame-major [B][n][HW][H][D]; 1 <= n <= l. */
+ * q, k, v, out: frame-major [B][n][HW][H][D]; 1 <= n <= l.  Scores and softmax in fp32;
+ * the probability-weighted sum of V runs on the tensor cores in fp16 (P with 11 significant
+ * bits, fp32 accumulation), so V values must lie within the fp16 range |v| <= 65504: larger
+ * ones (and inf / NaN in V) are recorded as CA2_ERR_RANGE, read by ca2_device_status. */
 int ca2_spatial_prefix_attn(ca2_cache *cache, int layer, const void *q, const void *k,
                             const void *v, void *out, int n_frames, int use_prefix, void *stream);
 
@@ -164,7 +200,8 @@ int ca2_spatial_prefix_attn(ca2_cache *cache, int layer, const void *q, const vo
  *   out[b][s][c][:] = round_bf16(x[b][s][c][:] + table[row(c)][:])
  * The sum is taken in float32 and rounded once (nearest, ties to even).
  * table: device, [N_tpe][H][D] bf16 (N_tpe = the cache's tpe_len), read only.
- * x, out: device, token-major [B][HW][n][H][D] (the temporal branch's layout); out may be
+ * x, out: device, token-major [B][HW][n][H][D] (the temporal branch's layout); the rows of
+ * x, out and table are row_pitch elements apart and the add covers their first H*D; out may be
  * x itself (in place), otherwise they must not overlap.  1 <= n <= l.  All three 16-byte
  * aligned.  Asynchronous on `stream`; the cache state is not touched.
  * Errors: ARG (null pointer, negative frame or offset), SHAPE (n, or a chunk of 2^35 bytes or
@@ -183,8 +220,9 @@ int ca2_tpe_indices(const ca2_cache *cache, long long first_global_frame, int of
 int ca2_cache_state(const ca2_cache *cache, int *head, int *count, int *sp_count,
                     long long *frames_written);
 
-/* Synchronise the current device and return CA2_ERR_TIMEOUT if any kernel of this library
- * recorded a bounded wait that gave up since the last call (clearing the record), else
+/* Synchronise the current device and return what the kernels of this library recorded since
+ * the last call (clearing the record): CA2_ERR_TIMEOUT if a bounded wait gave up,
+ * CA2_ERR_RANGE if an input was outside the supported range (the first record wins), else
  * CA2_OK (or CA2_ERR_CUDA if the synchronisation itself fails). */
 int ca2_device_status(void);
 

@@ -7,14 +7,20 @@ import numpy as np
 import oracle
 from ca2_synth import Generator, Workload, bf16_to_f32
 
-# Tolerance for floating-point outputs (bf16 inputs, fp32 softmax and accumulation,
-# bf16 output): relative L2 5e-3, and max-abs 2e-2 on the error beyond the output format's
-# own rounding radius.  The outputs are bf16 by contract, and bf16 rounding alone moves a
-# value of magnitude in [2^e, 2^(e+1)) by up to 2^(e-8) (0.0156 in [4, 8), 0.031 in
-# [8, 16)), which no bf16-output kernel can avoid; that radius is taken off before the
-# max-abs bound applies.  Values below 1 in magnitude have a radius under 0.002.
+# Tolerance for floating-point outputs (bf16 inputs, fp32 softmax and accumulation, bf16
+# output): max-abs 2e-2 and relative L2 5e-3, as stated for the path.  The max-abs bound is
+# applied to the raw error of every element whose exact value is below 8 in magnitude.  At 8
+# and above, rounding to bf16 alone can move a value by up to 2^(e-8) >= 0.031 (half an ulp
+# of 8 significant bits), more than the bound itself, so there the bound applies to the error
+# beyond that radius; such elements are counted and reported with the raw errors
+# (PARITY_LOG, printed at the end of the session by tests/conftest.py).
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
+BIG = 8.0
+
+# (label, raw max-abs, raw max-abs where |ref| < BIG, elements with |ref| >= BIG, elements
+# checked, rel-L2) per checked call
+PARITY_LOG = []
 
 
 def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
@@ -22,6 +28,13 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     ax = np.abs(x)
     e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
     return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
+def f16_bits_of_bf16(bits: np.ndarray) -> np.ndarray:
+    """The fp16 bit patterns of bf16 values (numpy's float32 -> float16 conversion rounds to
+    nearest even; it is exact for bf16 values within the fp16 range): the spatial cache keeps
+    its V in this form."""
+    return bf16_to_f32(bits).astype(np.float16).view(np.uint16)
 
 
 def to_dev(bits: np.ndarray):
@@ -40,17 +53,24 @@ def token_major(x: np.ndarray) -> np.ndarray:
 
 
 def check_close(got_bits: np.ndarray, ref: np.ndarray, what: str = ""):
-    """Returns (raw max-abs, max-abs beyond the bf16 output rounding, rel-L2)."""
+    """Assert the stated tolerance; returns (raw max-abs, elements with |ref| >= 8, rel-L2)."""
     got = bf16_to_f32(got_bits).astype(np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.isfinite(got).all(), "%s: non-finite output" % what
     err = np.abs(got - ref)
-    max_abs = float(err.max()) if err.size else 0.0
-    excess = float((err - bf16_half_ulp(ref)).max()) if err.size else 0.0
+    if not err.size:
+        return 0.0, 0, 0.0
+    big = np.abs(ref) >= BIG
+    n_big = int(big.sum())
+    max_abs = float(err.max())
+    small = float(err[~big].max()) if n_big < err.size else 0.0
+    excess = float((err[big] - bf16_half_ulp(ref[big])).max()) if n_big else 0.0
     rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
-    assert excess <= MAX_ABS and rel <= REL_L2, \
-        "%s: max-abs %.3g (beyond bf16 output rounding %.3g) rel-L2 %.3g" % (what, max_abs, excess, rel)
-    return max_abs, excess, rel
+    PARITY_LOG.append((what, max_abs, small, n_big, int(err.size), rel))
+    assert small <= MAX_ABS and excess <= MAX_ABS and rel <= REL_L2, \
+        "%s: max-abs %.3g where |ref| < %g; %d elements at |ref| >= %g with %.3g beyond bf16 rounding; " \
+        "rel-L2 %.3g" % (what, small, BIG, n_big, BIG, excess, rel)
+    return max_abs, n_big, rel
 
 
 class Loop:
@@ -78,12 +98,12 @@ class Loop:
         pk, pv = self.rings[layer].prefix()
         if units is None:
             ref = oracle.temporal_attn(q, k, v, pk, pv)
-            self.stats.append(("temporal", len(pk), n) + check_close(got, ref, "temporal P_k=%d" % len(pk)))
+            self.stats.append(("temporal", len(pk), n) + check_close(got, ref, "%s temporal" % self.wl.name))
         else:
             ref = oracle.temporal_attn(q, k, v, pk, pv, units=units)
             wl = self.wl
             g = got.transpose(0, 2, 3, 1, 4).reshape(wl.batch * wl.hw * wl.heads, n, wl.head_dim)[units]
-            self.stats.append(("temporal", len(pk), n) + check_close(g, ref, "temporal(sampled)"))
+            self.stats.append(("temporal", len(pk), n) + check_close(g, ref, "%s temporal" % self.wl.name))
         return got
 
     def spatial(self, layer, q, k, v, use_prefix, units=None):
@@ -98,12 +118,12 @@ class Loop:
             sk, sv, rep = [], [], self.wl.p_spatial + 1
         if units is None:
             ref = oracle.spatial_attn(q, k, v, sk, sv, repeat=rep)
-            self.stats.append(("spatial", len(sk), n) + check_close(got, ref, "spatial n_sp=%d" % len(sk)))
+            self.stats.append(("spatial", len(sk), n) + check_close(got, ref, "%s spatial" % self.wl.name))
         else:
             ref = oracle.spatial_attn(q, k, v, sk, sv, repeat=rep, units=units)
             wl = self.wl
             g = got.transpose(0, 1, 3, 2, 4).reshape(wl.batch * n * wl.heads, wl.hw, wl.head_dim)[units]
-            self.stats.append(("spatial", len(sk), n) + check_close(g, ref, "spatial(sampled)"))
+            self.stats.append(("spatial", len(sk), n) + check_close(g, ref, "%s spatial" % self.wl.name))
         return got
 
     # -- cache-writing stage ------------------------------------------------------------
@@ -133,7 +153,8 @@ class Loop:
                 sk = to_bits(self.cache.spatial(L, 0))
                 sv = to_bits(self.cache.spatial(L, 1))
                 for j, g in enumerate(ring.spatial_ids):
-                    assert np.array_equal(sk[j], ring.sk[g]) and np.array_equal(sv[j], ring.sv[g])
+                    assert np.array_equal(sk[j], ring.sk[g]), "spatial K frame %d" % g
+                    assert np.array_equal(sv[j], f16_bits_of_bf16(ring.sv[g])), "spatial V frame %d (fp16)" % g
 
     def tpe_check(self, n):
         g0 = self.rings[0].frames_written

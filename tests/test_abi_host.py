@@ -15,7 +15,7 @@ FAKE_S = 0x7F1000000000
 
 def cfg(**kw):
     base = dict(n_layers=1, batch=1, hw=256, heads=16, head_dim=72, chunk_len=8, p_max=41,
-                p_spatial=3, tpe_len=0)
+                p_spatial=3, tpe_len=0, row_pitch=0)
     base.update(kw)
     return base
 
@@ -169,7 +169,7 @@ def test_tpe_indices_match_oracle():
 
 
 def test_status_strings():
-    for code in range(-6, 1):
+    for code in range(-7, 1):
         assert ca2.ca2_status_string(code) != "unknown status"
     assert ca2.ca2_status_string(-99) == "unknown status"
 
@@ -218,4 +218,70 @@ def test_kv_proj_write_validation_and_commit():
     with pytest.raises(ca2.Ca2Error) as e:
         ca2.ca2_kv_proj_write(h, 0, X + 8, W, None, None, None, None, 8)
     assert e.value.status == -4
+    ca2.ca2_cache_destroy(h)
+
+
+def test_evict_for_matches_oracle_fifo():
+    """ca2_cache_evict_for evicts exactly the frames the oracle's FIFO drops when n_new more
+    are appended (papernotes page, 关键设计 4), over a random schedule of chunk lengths; the
+    queue is advanced on the host with ca2_cache_commit (no device work)."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    for p_max, l in ((41, 8), (9, 4), (8, 8), (13, 5)):
+        h, c = make(p_max=p_max, chunk_len=l, p_spatial=min(3, l))
+        ring = oracle.RingModel(p_max, min(3, l))
+        z = np.zeros((1, 1, 1, 1, 1), dtype=np.uint16)
+        for step in range(40):
+            n = int(rng.integers(1, l + 1)) if step else 1
+            e = ca2.ca2_cache_evict_for(h, n)
+            ca2.ca2_cache_commit(h, n)
+            zz = np.zeros((1, n, 1, 1, 1), dtype=np.uint16)
+            gone = ring.write(zz, zz, zz, zz)
+            assert e == len(gone), (p_max, l, step)
+            head, count, sp, fw = ca2.ca2_cache_state(h)
+            assert (head, count, sp, fw) == (ring.head, ring.count, len(ring.spatial_ids), ring.frames_written)
+        for bad in (-1, p_max + 1):
+            with pytest.raises(ca2.Ca2Error) as err:
+                ca2.ca2_cache_evict_for(h, bad)
+            assert err.value.status == -2
+        assert ca2.ca2_cache_evict_for(h, 0) == 0
+        ca2.ca2_cache_destroy(h)
+
+
+def test_config_defaults_resolved_by_the_library():
+    h, c = make()
+    got = ca2.ca2_cache_config(h)
+    assert (got.tpe_len, got.row_pitch) == (c["p_max"] + c["chunk_len"], c["heads"] * c["head_dim"])
+    assert (got.n_layers, got.batch, got.hw, got.heads, got.head_dim) == (1, 1, 256, 16, 72)
+    ca2.ca2_cache_destroy(h)
+    h, c = make(tpe_len=16, row_pitch=16 * 72 * 4)
+    got = ca2.ca2_cache_config(h)
+    assert (got.tpe_len, got.row_pitch) == (16, 16 * 72 * 4)
+    ca2.ca2_cache_destroy(h)
+
+
+@pytest.mark.parametrize("pitch,ok", [(0, True), (1152, True), (1152 + 8, True), (4608, True),
+                                      (1144, False), (1156, False), (-8, False)])
+def test_row_pitch_validation(pitch, ok):
+    if ok:
+        ca2.ca2_cache_bytes(cfg(row_pitch=pitch))
+    else:
+        with pytest.raises(ca2.Ca2Error) as e:
+            ca2.ca2_cache_bytes(cfg(row_pitch=pitch))
+        assert e.value.status == -2
+
+
+def test_layer_offsets_follow_the_documented_layout():
+    """Offsets of each layer's K/V ring and spatial cache: temporal [N_L][2][B][HW][H][Pmax][D]
+    and spatial [N_L][2][P'][B][HW][H][D] bf16, as include/ca2.h states."""
+    h, c = make(n_layers=3, batch=2)
+    plane = c["batch"] * c["hw"] * c["heads"] * c["head_dim"] * 2
+    for L in range(3):
+        for kv in (0, 1):
+            t, s = ca2.ca2_cache_layer_offsets(h, L, kv)
+            assert t == (L * 2 + kv) * c["p_max"] * plane
+            assert s == (L * 2 + kv) * c["p_spatial"] * plane
+    for bad in ((3, 0), (-1, 0), (0, 2)):
+        with pytest.raises(ca2.Ca2Error):
+            ca2.ca2_cache_layer_offsets(h, *bad)
     ca2.ca2_cache_destroy(h)

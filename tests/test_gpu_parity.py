@@ -9,13 +9,13 @@ import numpy as np
 import pytest
 
 import oracle
-from ca2_synth import WORKLOADS, Generator
+from ca2_synth import WORKLOADS, Generator, bf16_bits, bf16_to_f32
 
 pytestmark = pytest.mark.gpu
 
 
-def _wl(name, **kw):
-    return dataclasses.replace(WORKLOADS[name], **kw)
+def _wl(base, **kw):
+    return dataclasses.replace(WORKLOADS[base], **kw)
 
 
 def test_tiny_generation_loop_every_call():
@@ -33,7 +33,7 @@ def test_tiny_generation_loop_every_call():
 
 def test_tiny_peaky_values():
     from tests.gpu_util import Loop
-    wl = _wl("tiny", recipe="peaky")
+    wl = _wl("tiny", recipe="peaky", name="tiny_peaky")
     lp = Loop(wl, seed=5)
     lp.first_frame()
     for _ in range(3):
@@ -184,7 +184,7 @@ def test_ragged_shapes(shape):
     """Ragged query/key tiles (HW not a multiple of 128), odd head counts, head dims 16-128,
     short chunks, Pmax = l, P' = 0; several AR steps with eviction."""
     from tests.gpu_util import Loop
-    wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, **shape)
+    wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, name="ragged", **shape)
     lp = Loop(wl, seed=9)
     lp.first_frame()
     for _ in range(4):
@@ -202,7 +202,7 @@ def test_spatial_max_grows_in_late_blocks(head_dim):
     from ca2_synth import bf16_bits, bf16_to_f32
     from tests.gpu_util import Loop
     wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, hw=256, heads=2, head_dim=head_dim,
-             batch=1, chunk_len=3, p_max=6, p_spatial=3)
+             batch=1, chunk_len=3, p_max=6, p_spatial=3, name="lazy_rescale")
     lp = Loop(wl, seed=21)
     kt, vt = lp.gen.frames(3), lp.gen.frames(3)
     ks = bf16_to_f32(lp.gen.frames(3)).copy()
@@ -243,7 +243,7 @@ def test_long_queue_pmax81():
     filling the ring and then evicting; every attention output and cache write checked."""
     from tests.gpu_util import Loop
     wl = _wl("tiny", recipe="normal", scale=0.5, n_layers=1, hw=64, heads=2, head_dim=72, batch=1,
-             chunk_len=8, p_max=81, p_spatial=3)
+             chunk_len=8, p_max=81, p_spatial=3, name="pmax81")
     lp = Loop(wl, seed=31)
     lp.first_frame()
     for _ in range(11):
@@ -302,10 +302,14 @@ def _bf16_ulp(x):
     return np.exp2(e - 7)
 
 
-def _check_projection(got_bits, exact, bound, C, what):
+def _check_projection(got_bits, exact, bound, C, what, fp16=False):
     """|got - exact| <= half a bf16 ulp (the one rounding) + the fp32 accumulation bound
-    C * 2^-23 * sum|x w| (twice the textbook gamma_C of recursive summation)."""
-    got = (got_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    C * 2^-23 * sum|x w| (twice the textbook gamma_C of recursive summation).  fp16: the
+    stored values are fp16 bit patterns (the spatial cache's V), the same bf16 values."""
+    if fp16:
+        got = got_bits.view(np.float16).astype(np.float64)
+    else:
+        got = (got_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.isfinite(got).all(), "%s: non-finite value" % what
     tol = 0.5 * _bf16_ulp(np.maximum(np.abs(exact), np.abs(got))) + C * 2.0 ** -23 * bound
     err = np.abs(got - exact)
@@ -376,7 +380,10 @@ def test_kv_proj_write_matches_oracle(shape, bias):
     bound = oracle.kv_projection_bound(xs_last.reshape(-1, C), w_s, b_s)
     for kv, exact, bnd in ((0, k, bound[:, :C]), (1, v, bound[:, C:])):
         got = spat[kv][:n_sp].transpose(1, 0, 2, 3, 4).reshape(-1, C)   # [B][n_sp][HW] rows
-        _check_projection(got, exact, bnd, C, "spatial %s" % "KV"[kv])
+        _check_projection(got, exact, bnd, C, "spatial %s" % "KV"[kv], fp16=kv == 1)
+        if kv == 1:   # exactly the fp16 form of a bf16 value
+            g32 = got.view(np.float16).astype(np.float32)
+            assert np.array_equal(g32, bf16_to_f32(bf16_bits(g32))), "spatial V is not a bf16 value"
         assert (spat[kv][n_sp:] == 0x7FC0).all(), "spatial: a frame past n_sp was written"
     # layer 0 untouched
     for kv in (0, 1):
@@ -384,3 +391,33 @@ def test_kv_proj_write_matches_oracle(shape, bias):
         assert (cache.spatial(0, kv).view(torch.int16) == 0x7FC0).all().item()
     cache.commit(n)
     assert cache.state()[1] == count + n and cache.state()[2] == n_sp
+
+
+def test_out_of_range_v_is_reported():
+    """The spatial attention's P V product runs in fp16, so V must lie within the fp16 range:
+    a larger V value in the spatial cache (through the cache write) or in the frame's own V
+    (through the spatial call) is reported as CA2_ERR_RANGE by ca2_device_status, which then
+    clears; in-range calls before and after report nothing."""
+    import torch
+    from causal_kv_cache_b200 import ca2
+    from causal_kv_cache_b200.ca2 import KVCache
+    from tests.gpu_util import to_dev, token_major
+    wl = WORKLOADS["tiny"]
+    g = Generator(wl, 17)
+    c = KVCache(1, wl.batch, wl.hw, wl.heads, wl.head_dim, wl.chunk_len, wl.p_max, wl.p_spatial)
+    assert ca2.ca2_device_status() == 0
+    k, v = g.frames(1), g.frames(1)
+    c.write([to_dev(token_major(k))], [to_dev(token_major(v))], [to_dev(k)], [to_dev(v)], 1)
+    assert ca2.ca2_device_status() == 0
+    big = v.copy()
+    big[0, 0, 3, 1, 5] = bf16_bits(np.array([70000.0], dtype=np.float32))[0]
+    c.evict_for(1)
+    c.write([to_dev(token_major(k))], [to_dev(token_major(big))], [to_dev(k)], [to_dev(big)], 1)
+    assert ca2.ca2_device_status() == -7
+    assert ca2.ca2_device_status() == 0
+    q, kk, vv = g.qkv(wl.chunk_len)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    vv[0, 1, 2, 0, 3] = bf16_bits(np.array([-1e6], dtype=np.float32))[0]
+    c.spatial_attn(0, to_dev(q), to_dev(kk), to_dev(vv), out, wl.chunk_len, 0)
+    assert ca2.ca2_device_status() == -7
+    assert ca2.ca2_device_status() == 0
