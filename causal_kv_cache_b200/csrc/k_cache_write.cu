@@ -33,7 +33,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 // blockIdx.y = (layer, tensor): tensor 0/1 = temporal K/V, 2/3 = spatial K/V.
 //   temporal: chunk [B][HW][n][H][D] -> ring [B][HW][H][Pmax][D]; (token, j, h) -> slot (slot0 + j) mod Pmax
 //   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
-//             (K copied, V converted to fp16)
+//   (K copied, V converted to fp16)
 // (source rows are src_row_vec 16-byte vectors apart, of which the first row_vec are copied)
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
@@ -84,10 +84,10 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
             v[i] = ld_stream(src + so[i]);
         }
     }
-    if (tensor == 3) {
-        // the spatial cache keeps V in fp16, the operand type of the spatial attention's P V
-        // product: the exact value of each bf16 element within the fp16 range; elements
-        // beyond it (|v| >= 65536, inf, NaN) are recorded as a range error
+    if (tensor & 1) {
+        // both caches keep V in fp16, the operand type of the attention's P V products: the
+        // exact value of each bf16 element within the fp16 range; elements beyond it
+        // (|v| >= 65536, inf, NaN) are recorded as a range error
         uint32_t vmax = 0;
 #pragma unroll
         for (int i = 0; i < kVecPerThread; ++i) {

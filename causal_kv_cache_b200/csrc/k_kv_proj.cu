@@ -261,9 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
                     w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + b8[2], __uint_as_float(v[8 * q + 3]) + b8[3]);
                     w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) + b8[4], __uint_as_float(v[8 * q + 5]) + b8[5]);
                     w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) + b8[6], __uint_as_float(v[8 * q + 7]) + b8[7]);
-                    if (d.spatial && kv) {
-                        // the spatial cache keeps V in fp16: the exact value of the bf16 result
-                        // within the fp16 range, larger values recorded as a range error
+                    if (kv) {
+                        // both caches keep V in fp16: the exact value of the bf16 result within
+                        // the fp16 range, larger values recorded as a range error
                         vmax = __vmaxu2(vmax, abs_max4(w.x, w.y, w.z, w.w));
                         w = make_uint4(pack_f16x2(bf16_lo(w.x), bf16_hi(w.x)), pack_f16x2(bf16_lo(w.y), bf16_hi(w.y)),
                                        pack_f16x2(bf16_lo(w.z), bf16_hi(w.z)), pack_f16x2(bf16_lo(w.w), bf16_hi(w.w)));

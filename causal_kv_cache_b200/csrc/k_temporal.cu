@@ -32,9 +32,10 @@
 //     products use mma.sync on registers: S^T = K Q^T (keys on M, the 8 queries on N),
 //     then O^T += V^T P^T.  Each lane owns the same two query columns in both
 //     accumulators, so the online-softmax rescale is lane-local; movmatrix turns P^T
-//     into the B operand and O^T back into rows for the stores.  P enters the product as
-//     two bf16 parts (P rounded, then the remainder rounded), so the probabilities carry
-//     16 significant bits rather than 8.  The reference max of the exponentials moves
+//     into the B operand and O^T back into rows for the stores.  P V runs in fp16 (P with
+//     11 significant bits rather than bf16's 8): the ring keeps V in fp16 (converted
+//     exactly when written), and the chunk's own V is converted in registers.  The
+//     reference max of the exponentials moves
 //     only when a score exceeds it by more than 2^8 (one warp vote per stage; the max
 //     reduction and the rescale run only then), which leaves each softmax row unchanged
 //     after normalisation.
@@ -99,6 +100,17 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma16816_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// bf16 pair -> fp16 pair (exact within the fp16 range)
+__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t w) { return pack_f16x2(bf16_lo(w), bf16_hi(w)); }
 __device__ __forceinline__ void mma1688(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0)
 {
     asm volatile(
@@ -317,6 +329,7 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
         const int q0 = 2 * (lane & 3);        // this lane's two query columns: q0, q0 + 1
         const int krow = lane >> 2;            // this lane's key rows in a stage: krow, krow + 8
         const float neg_inf = __int_as_float(0xff800000);
+        uint32_t vmax = 0;                     // per-half max of |v| bits of the chunk's V
         int stage = 0;
         for (int li = 0;; ++li) {
             const int qs = li & 1;
@@ -441,22 +454,15 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         acc[t][3] *= al1;
                     }
                 }
-                // probabilities as a bf16 pair hi + lo (hi = P rounded to bf16, lo = the rest
-                // rounded to bf16: 16 significant bits between them), each multiplied by V^T on
-                // the tensor core; a single bf16 P would carry up to 2^-9 relative error into
-                // every output, the same order as the output's own rounding
+                // probabilities in fp16 (11 significant bits; bf16 P would carry up to 2^-9
+                // relative error into every output, the order of the output's own rounding);
+                // the normaliser sums the fp32 values (2^-12 from the rounded ones)
                 const float e0 = ex2(sc[0] - m_run[0]), e1 = ex2(sc[1] - m_run[1]);
                 const float e2 = ex2(sc[2] - m_run[0]), e3 = ex2(sc[3] - m_run[1]);
-                const uint32_t x0 = pack_bf16x2(e0, e1);
-                const uint32_t x1 = pack_bf16x2(e2, e3);
-                const uint32_t r0 = pack_bf16x2(e0 - bf16_lo(x0), e1 - bf16_hi(x0));
-                const uint32_t r1 = pack_bf16x2(e2 - bf16_lo(x1), e3 - bf16_hi(x1));
                 l_part[0] += e0 + e2;
                 l_part[1] += e1 + e3;
-                const uint32_t pb0 = movm_t(x0);
-                const uint32_t pb1 = movm_t(x1);
-                const uint32_t pl0 = movm_t(r0);
-                const uint32_t pl1 = movm_t(r1);
+                const uint32_t pb0 = movm_t(pack_f16x2(e0, e1));
+                const uint32_t pb1 = movm_t(pack_f16x2(e2, e3));
                 // O^T += V^T P^T, 16 head dims per m-tile
 #pragma unroll
                 for (int t = 0; t < DT; ++t) {
@@ -465,14 +471,22 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4_t(vbase + (uint32_t)((lane & 7) + 8 * (j >> 1)) * row + (uint32_t)(16 * t + 8 * (j & 1)) * 2u,
                                   a0, a1, a2, a3);
-                        mma16816(acc[t], a0, a1, a2, a3, pb0, pb1);
-                        mma16816(acc[t], a0, a1, a2, a3, pl0, pl1);
+                        if (st == 0) {
+                            // the chunk's own V arrives as bf16; its key rows 8..15 (a2, a3) are
+                            // frames past the chunk (n <= 8), zero-filled, the same in fp16
+                            vmax = __vmaxu2(vmax, abs_max4(a0, a1, 0u, 0u));
+                            a0 = bf2_to_h2(a0), a1 = bf2_to_h2(a1);
+                        }
+                        mma16816_f16(acc[t], a0, a1, a2, a3, pb0, pb1);
                     } else {
                         uint32_t a0, a2;
                         ldsm_x2_t(vbase + (uint32_t)((lane & 7) + 8 * ((lane >> 3) & 1)) * row + (uint32_t)(16 * t) * 2u,
                                   a0, a2);
-                        mma16816(acc[t], a0, 0u, a2, 0u, pb0, pb1);
-                        mma16816(acc[t], a0, 0u, a2, 0u, pl0, pl1);
+                        if (st == 0) {
+                            vmax = __vmaxu2(vmax, abs_max4(a0, 0u, 0u, 0u));
+                            a0 = bf2_to_h2(a0);
+                        }
+                        mma16816_f16(acc[t], a0, 0u, a2, 0u, pb0, pb1);
                     }
                 }
                 __syncwarp();
@@ -502,6 +516,8 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                 }
             }
         }
+        // a chunk V beyond the fp16 range (|v| >= 65536, inf, NaN): a range error
+        if ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u) record_status(kStatusRange);
     }
 }
 

@@ -35,9 +35,9 @@
  *   temporal: [N_L][2][B][HW][H][Pmax][D]   (index 0 = K ring, 1 = V ring; token-major and
  *                                            head-major within a token: one head's Pmax
  *                                            slots are contiguous)
- *   spatial : [N_L][2][P'][B][HW][H][D]     (K in bf16; V in fp16, the operand type of the
- *                                            spatial attention's P V product: each bf16 value
- *                                            converted exactly, |v| <= 65504)
+ *   spatial : [N_L][2][P'][B][HW][H][D]
+ * K is stored in bf16 and V in fp16, the operand type of the attention's P V products (each
+ * bf16 value converted exactly; |v| <= 65504).
  * The i-th oldest queued frame (i = 0 .. count-1) is in ring slot (head + i) mod Pmax;
  * spatial slot j (j < sp_count) holds the j-th of the last sp_count frames written,
  * oldest first.  Slots that hold no queued frame may contain anything: they are masked,
@@ -128,8 +128,8 @@ int ca2_cache_evict_for(ca2_cache *cache, int n_new, int *evicted);
  * frames j = 0..n-1 of k_t[L], v_t[L] are copied into ring slots
  * (head + count + j) mod Pmax; then the spatial cache of layer L is overwritten with the
  * last min(P', n) frames of k_s[L], v_s[L].  count += n.  One kernel launch for all
- * layers; a bit-exact copy, except that the spatial V is stored as fp16 (the same values;
- * |v| >= 65536, inf or NaN there is recorded as CA2_ERR_RANGE, read by ca2_device_status).
+ * layers; a bit-exact copy, except that V is stored as fp16 (the same values; |v| >= 65536,
+ * inf or NaN there is recorded as CA2_ERR_RANGE, read by ca2_device_status).
  * k_t[L], v_t[L] are token-major [B][HW][n][H][D]; k_s[L],
  * v_s[L] are frame-major [B][n][HW][H][D].  k_t, v_t, k_s, v_s are HOST arrays of N_L
  * device pointers (k_s, v_s may be NULL when P' = 0); their rows are row_pitch elements
@@ -152,8 +152,7 @@ int ca2_cache_write(ca2_cache *cache, const void *const *k_t, const void *const 
  * [2C][Cin] row-major, row o = output channel o (K channels 0..C-1 as (head, dim), then V);
  * b_t, b_s: [2C] or NULL for no bias.  All bf16, device memory, 16-byte aligned.  fp32
  * accumulation on the tensor cores, then the bias, then one rounding to bf16 (nearest,
- * ties to even); the spatial V is stored as the fp16 of that bf16 value (see the cache
- * layout above).  x_s, w_s, b_s are not read when n_sp = 0 (may be NULL).
+ * ties to even); V is stored as the fp16 of that bf16 value (see the cache layout above).  x_s, w_s, b_s are not read when n_sp = 0 (may be NULL).
  * The queue does not advance: after this call for every layer, call ca2_cache_commit(n)
  * (evict first, as for ca2_cache_write).  1 <= n <= chunk_len and count + n <= Pmax, else
  * CA2_ERR_SHAPE / CA2_ERR_CAPACITY.  Asynchronous on `stream`. */
@@ -173,7 +172,9 @@ int ca2_cache_commit(ca2_cache *cache, int n_frames);
  * queued frames are all visible, so their order does not matter).  The cache is only
  * read.  q, k, v, out: token-major [B][HW][n][H][D] device pointers; out must not
  * overlap the inputs.  1 <= n <= l.  fp32 softmax and accumulation, bf16 output (round
- * to nearest even). */
+ * to nearest even).  The probability-weighted sum of V runs in fp16 (P with 11 significant
+ * bits), so V must lie within |v| <= 65504: a larger chunk V (or inf / NaN) is recorded as
+ * CA2_ERR_RANGE, read by ca2_device_status. */
 int ca2_temporal_attn(ca2_cache *cache, int layer, const void *q, const void *k, const void *v,
                       void *out, int n_frames, void *stream);
 

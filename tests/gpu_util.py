@@ -32,8 +32,8 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
 
 def f16_bits_of_bf16(bits: np.ndarray) -> np.ndarray:
     """The fp16 bit patterns of bf16 values (numpy's float32 -> float16 conversion rounds to
-    nearest even; it is exact for bf16 values within the fp16 range): the spatial cache keeps
-    its V in this form."""
+    nearest even; it is exact for bf16 values within the fp16 range): both caches keep their
+    V in this form."""
     return bf16_to_f32(bits).astype(np.float16).view(np.uint16)
 
 
@@ -148,7 +148,8 @@ class Loop:
             for g in ring.queue:
                 slot = ring.slot_of(g)
                 assert np.array_equal(rk[:, :, :, slot], ring.k[g]), "K ring slot %d (frame %d)" % (slot, g)
-                assert np.array_equal(rv[:, :, :, slot], ring.v[g]), "V ring slot %d (frame %d)" % (slot, g)
+                assert np.array_equal(rv[:, :, :, slot], f16_bits_of_bf16(ring.v[g])), \
+                    "V ring slot %d (frame %d, fp16)" % (slot, g)
             if self.wl.p_spatial:
                 sk = to_bits(self.cache.spatial(L, 0))
                 sv = to_bits(self.cache.spatial(L, 1))
