@@ -39,6 +39,20 @@ WORKLOAD = dict(batch=1, hw=256, heads=16, head_dim=72, chunk_len=8, p_max=41, p
                 n_layers=28, denoise_steps=50)
 WORKLOAD_NAME = ("Open-Sora-shaped attention layer, Pmax=41 full queue (steady-state AR step of the "
                  "80-frame run), 28 per-block caches")
+# The Ca2-VDM settings timed by --config (Open-Sora v1.0 backbone: C = 1152 in 16 heads of 72,
+# chunk l = 8, P' = 3, T = 50): one AR step at the configuration's steady state, every block's
+# queue at Pmax.  The default is os_p41.
+CONFIGS = {
+    "os_p41": dict(batch=1, hw=256, p_max=41, name=WORKLOAD_NAME),
+    "os_p25": dict(batch=1, hw=256, p_max=25,
+                   name="Open-Sora-shaped attention layer, Pmax=25 full queue (P in {1, 9, 17, 25}), "
+                        "28 per-block caches"),
+    "os_28blk_b4": dict(batch=4, hw=256, p_max=41,
+                        name="attention sub-path of the 28-block backbone, B=4 videos, Pmax=41 full queue"),
+    "hires": dict(batch=2, hw=1024, p_max=41,
+                  name="512x512 video (32x32 = 1024 tokens/frame), B=2, Pmax=41 full queue, "
+                       "spatial map 1024 x 4096"),
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -48,14 +62,17 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ca2", choices=["ca2", "reference"])
+    ap.add_argument("--config", default="os_p41", choices=sorted(CONFIGS),
+                    help="which Ca2-VDM setting one step runs (default os_p41, the Pmax=41 layer)")
     ap.add_argument("--layers", type=int, default=WORKLOAD["n_layers"])
     ap.add_argument("--denoise", type=int, default=WORKLOAD["denoise_steps"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="step", choices=["step", "recompute", "per-timestep"],
+    ap.add_argument("--mode", default="step", choices=["step", "recompute", "per-timestep", "cpu-baseline"],
                     help="step: the timed AR step (default); recompute: cached vs recompute-from-scratch "
                          "attention per denoising step along the 80-frame run; per-timestep: one shared "
-                         "cache vs one cache per denoising step (memory and AR-step time)")
+                         "cache vs one cache per denoising step (memory and AR-step time); cpu-baseline: "
+                         "the oracle per call, one thread and all host threads, at every queue length")
     return ap.parse_args()
 
 
@@ -166,7 +183,9 @@ def run_ca2(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
-    W = dict(WORKLOAD, n_layers=args.layers, denoise_steps=args.denoise)
+    cfg = CONFIGS[args.config]
+    W = dict(WORKLOAD, n_layers=args.layers, denoise_steps=args.denoise,
+             **{k: cfg[k] for k in ("batch", "hw", "p_max")})
     B, HW, H, D, l, PM, PS = (W[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max", "p_spatial"))
     NL, T = W["n_layers"], W["denoise_steps"]
     plane = B * HW * H * D
@@ -188,8 +207,11 @@ def run_ca2(args):
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
 
-    # fill the queue: first frame + 5 chunks -> 41 frames, spatial cache 3
-    for n in (1, 8, 8, 8, 8, 8):
+    # fill the queue: the first frame, then chunks of l until it holds Pmax frames
+    fills = [1]
+    while 1 + l * (len(fills) - 1) < PM:
+        fills.append(l)
+    for n in fills:
         kt = [rnd(n, True) for _ in range(NL)]
         vt = [rnd(n, True) for _ in range(NL)]
         ks = [rnd(n) for _ in range(NL)]
@@ -206,7 +228,7 @@ def run_ca2(args):
     P = [{k: ptr(v) for k, v in d.items()} for d in inp]
     SO = [ptr(t) for t in so]
     TO = [ptr(t) for t in to]
-    g0 = [1 + 8 * 5]
+    g0 = [1 + l * (len(fills) - 1)]
     # device input/output sets the step can run on (the end-to-end run adds a second one so
     # that copies overlap compute); cur[0] selects the set the next step captures
     sets = [dict(P=P, SO=SO, TO=TO)]
@@ -427,7 +449,7 @@ def run_ca2(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.49) bf16 Q/K/V; no weights needed)",
-        "config": {"workload": WORKLOAD_NAME, "batch": B, "tokens_per_frame": HW, "heads": H,
+        "config": {"workload": cfg["name"], "config": args.config, "batch": B, "tokens_per_frame": HW, "heads": H,
                    "head_dim": D, "chunk_len": l, "p_max": PM, "p_spatial": PS, "blocks": NL,
                    "denoise_steps": T, "queue_len": PM, "parallelism": "replica per GPU (dp%d)" % world,
                    "l2": "inputs larger than L2: %d per-block caches and inputs, %.2f GB on the device"
@@ -581,6 +603,83 @@ def oracle_sample(budget_s: float):
 def cpu_baseline(budget_s: float):
     value, sample, cores, _ = oracle_sample(budget_s)
     return {"value": value, "unit": "query-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+
+def run_cpu_baseline(args):
+    """The fp64 oracle as a reported CPU baseline (never a target), on the machine's host cores.
+
+    Per call of the Open-Sora-shaped layer (B=1, HW=256, 16 x 72, l=8, P'=3) at every queue
+    length of the 80-frame run (P_k = 1, 9, ..., 41): temporal attention (B*HW*H units of 8
+    queries) and prefix-spatial attention (B*n*H frame-heads; n_sp = 1 at P_k = 1, else 3),
+    each timed on a bounded sample of units with one thread and with all threads and scaled
+    to the whole call.  Then one 512x512 (1024 tokens/frame, B = 2) prefix-spatial call on all
+    threads, from a sample of frame-heads, extrapolated to an AR step of T = 50 denoising calls
+    plus the cache-writing pass: an extrapolation, stated as such."""
+    rank, _, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from ca2_synth import Generator, WORKLOADS
+    oracle.build()
+    all_threads = oracle.num_threads()
+    wl = WORKLOADS["os_p41"]
+    gen = Generator(wl, 0)
+    q, k, v = gen.qkv(wl.chunk_len)
+    _, pk, pv = gen.qkv(wl.p_max)
+    H = wl.heads
+    t_units_call = wl.batch * wl.hw * H
+    s_units_call = wl.batch * wl.chunk_len * H
+
+    def timed(fn, min_s=0.3):
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= min_s:
+                return dt / reps
+
+    rows = []
+    for P in (1, 9, 17, 25, 33, 41):
+        prefix_k = [pk[:, i] for i in range(P)]
+        prefix_v = [pv[:, i] for i in range(P)]
+        n_sp = 1 if P == 1 else 3
+        sk, sv = prefix_k[-n_sp:], prefix_v[-n_sp:]
+        row = {"p_k": P, "n_sp": n_sp}
+        for label, threads, tu, su in (("1_thread", 1, 16, 1), ("all_threads", all_threads, 16 * all_threads,
+                                                                 max(1, min(s_units_call, all_threads)))):
+            oracle.set_num_threads(threads)
+            t_u = np.arange(tu)
+            s_u = np.arange(su)
+            tt = timed(lambda: oracle.temporal_attn(q, k, v, prefix_k, prefix_v, units=t_u))
+            ts = timed(lambda: oracle.spatial_attn(q, k, v, sk, sv, repeat=0, units=s_u))
+            row[label] = {"temporal_call_s": tt * t_units_call / tu, "spatial_call_s": ts * s_units_call / su,
+                          "temporal_sample_units": tu, "spatial_sample_units": su}
+        rows.append(row)
+    # 512x512: one prefix-spatial call (B=2, 8 frames, 16 heads: 256 frame-heads of 1024 x 4096)
+    hw = WORKLOADS["hires"]
+    hgen = Generator(hw, 0)
+    hq, hk, hv = hgen.qkv(hw.chunk_len)
+    _, hck, hcv = hgen.qkv(3)
+    oracle.set_num_threads(all_threads)
+    hs_units = np.arange(all_threads)
+    th = timed(lambda: oracle.spatial_attn(hq, hk, hv, [hck[:, i] for i in range(3)], [hcv[:, i] for i in range(3)],
+                                           repeat=0, units=hs_units), min_s=0.0)
+    units_call = hw.batch * hw.chunk_len * hw.heads
+    hires_call = th * units_call / len(hs_units)
+    oracle.set_num_threads(all_threads)
+    out = {
+        "impl": "oracle-cpu-baseline", "kind": "oracle", "cores": all_threads, "host_cpus": os.cpu_count(),
+        "precision": "f64 naive (two-pass softmax), gcc -O2, OpenMP over units",
+        "per_call": rows,
+        "hires_spatial": {"call_s_all_threads": hires_call, "sample_frame_heads": len(hs_units),
+                          "frame_heads_per_call": units_call,
+                          "ar_step_s_extrapolated": hires_call * 51,
+                          "note": "extrapolation: one call's time from a sample of frame-heads, times the "
+                                  "T = 50 denoising calls plus the cache-writing pass of one AR step"},
+    }
+    print(json.dumps(out))
 
 
 def run_reference(args):
@@ -811,6 +910,8 @@ def main():
         run_recompute(args)
     elif args.mode == "per-timestep":
         run_per_timestep(args)
+    elif args.mode == "cpu-baseline":
+        run_cpu_baseline(args)
     else:
         run_ca2(args)
 
