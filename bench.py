@@ -17,6 +17,14 @@ through one block's spatial + temporal attention, so a step counts (T+1) * 28 * 
 
 Under torchrun each rank runs the same step on its own GPU with its own caches (videos
 are independent; no data-path collective); value = all ranks' tokens / max rank time.
+
+  python bench.py --shard heads [...]
+
+splits the heads instead (tensor-parallel attention): rank r of N owns the contiguous heads
+ca2_head_shard gives it, keeps caches for those heads only and runs them on full-width
+activations through the row pitch, again with no collective on the path (attention never
+mixes heads); the whole job processes each step's tokens once (strong scaling).  On one
+process, --shard-world G --shard-rank r times rank r's share of a G-way split alone.
 """
 from __future__ import annotations
 
@@ -66,6 +74,13 @@ def parse():
                     help="which Ca2-VDM setting one step runs (default os_p41, the Pmax=41 layer)")
     ap.add_argument("--layers", type=int, default=WORKLOAD["n_layers"])
     ap.add_argument("--denoise", type=int, default=WORKLOAD["denoise_steps"])
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="none: every rank runs the whole step (replicas, weak scaling); heads: the ranks "
+                         "split the heads of every block (strong scaling)")
+    ap.add_argument("--shard-world", type=int, default=0,
+                    help="with --shard heads in a single process: the number of head groups to split into")
+    ap.add_argument("--shard-rank", type=int, default=0,
+                    help="with --shard-world: which group this process runs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="step", choices=["step", "recompute", "per-timestep", "cpu-baseline"],
@@ -186,24 +201,35 @@ def run_ca2(args):
     cfg = CONFIGS[args.config]
     W = dict(WORKLOAD, n_layers=args.layers, denoise_steps=args.denoise,
              **{k: cfg[k] for k in ("batch", "hw", "p_max")})
-    B, HW, H, D, l, PM, PS = (W[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max", "p_spatial"))
+    B, HW, H_all, D, l, PM, PS = (W[k] for k in ("batch", "hw", "heads", "head_dim", "chunk_len", "p_max",
+                                                  "p_spatial"))
     NL, T = W["n_layers"], W["denoise_steps"]
+    # heads this process runs: all of them, or its group of a head split (activations stay
+    # full width; the kernels get views at head h0 and the full row pitch)
+    if args.shard == "heads":
+        groups = world if world > 1 else max(1, args.shard_world)
+        grank = rank if world > 1 else args.shard_rank
+        h0, H = ca2.ca2_head_shard(H_all, groups, grank)
+    else:
+        groups, grank, h0, H = 1, 0, 0, H_all
+    sharded = args.shard == "heads"
+    hv = (lambda t: t[..., h0:h0 + H, :]) if sharded else (lambda t: t)
     plane = B * HW * H * D
     frame_bytes = plane * 2
-    cache = ca2.KVCache(NL, B, HW, H, D, l, PM, PS)
+    cache = ca2.KVCache(NL, B, HW, H, D, l, PM, PS, row_pitch=H_all * D if sharded else 0)
     g = torch.Generator(device=dev)
-    g.manual_seed(1234 + rank)
+    g.manual_seed(1234 + (0 if sharded else rank))      # the ranks of a head split share activations
 
     def rnd(n, token_major=False):
-        shape = (B, HW, n, H, D) if token_major else (B, n, HW, H, D)
+        shape = (B, HW, n, H_all, D) if token_major else (B, n, HW, H_all, D)
         return (torch.randn(shape, generator=g, device=dev) * 0.7).to(torch.bfloat16)
 
     # per-block inputs, reused across passes: spatial tensors frame-major [B][l][HW][H][D],
     # temporal tensors token-major [B][HW][l][H][D]
     inp = [dict(sq=rnd(l), sk=rnd(l), sv=rnd(l), tq=rnd(l, True), tk=rnd(l, True), tv=rnd(l, True))
            for _ in range(NL)]
-    so = [torch.empty((B, l, HW, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
-    to = [torch.empty((B, HW, l, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    so = [torch.empty((B, l, HW, H_all, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    to = [torch.empty((B, HW, l, H_all, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
     stream = torch.cuda.current_stream()
     sp = int(stream.cuda_stream)
 
@@ -217,14 +243,14 @@ def run_ca2(args):
         ks = [rnd(n) for _ in range(NL)]
         vs = [rnd(n) for _ in range(NL)]
         cache.evict_for(n)
-        cache.write(kt, vt, ks, vs, n, sp)
+        cache.write([hv(x) for x in kt], [hv(x) for x in vt], [hv(x) for x in ks], [hv(x) for x in vs], n, sp)
     torch.cuda.synchronize()
     assert cache.state()[1] == PM
 
     h = cache.handle
     tempo = ca2.ca2_temporal_attn
     spat = ca2.ca2_spatial_prefix_attn
-    ptr = lambda t: t.data_ptr()
+    ptr = lambda t: hv(t).data_ptr()
     P = [{k: ptr(v) for k, v in d.items()} for d in inp]
     SO = [ptr(t) for t in so]
     TO = [ptr(t) for t in to]
@@ -342,20 +368,29 @@ def run_ca2(args):
             continue
         (sp_den if kind == "den" else sp_self).append(a.elapsed_time(b_) / NL)
         tp_ms.append(b_.elapsed_time(c) / NL)
-    resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * plane) * 2 / 1e9
+    resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * HW * H_all * D) * 2 / 1e9
     launches_per_step = (T + 1) * NL * 2 + 1
     tokens_per_step = (T + 1) * NL * B * l * HW
-    value = whole_job_rate(tokens_per_step, args.steps, world, ms)
+    # query tokens the whole job moves through attention per step: every replica its own; a
+    # head split moves each token once over all ranks, and one group timed alone counts its
+    # heads' share
+    if not sharded:
+        job_tokens = tokens_per_step * world
+    elif world > 1:
+        job_tokens = tokens_per_step
+    else:
+        job_tokens = tokens_per_step * H / H_all
+    value = whole_job_rate(job_tokens, args.steps, 1, ms)
 
     # ---- cyclic TPE add (a next-row kernel, timed on its own, outside the step) ----
     # 28 launches (one per block's temporal input) in a CUDA graph, replayed 5 times
-    tpe_table = (torch.randn((cache.tpe_len, H, D), generator=g, device=dev) * 0.7).to(torch.bfloat16)
-    tpe_out = [torch.empty((B, HW, l, H, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
+    tpe_table = (torch.randn((cache.tpe_len, H_all, D), generator=g, device=dev) * 0.7).to(torch.bfloat16)
+    tpe_out = [torch.empty((B, HW, l, H_all, D), dtype=torch.bfloat16, device=dev) for _ in range(NL)]
     gt = torch.cuda.CUDAGraph()
     with torch.cuda.stream(cap):
         gt.capture_begin()
         for L in range(NL):
-            ca2.ca2_tpe_add(h, g0[0], 0, tpe_table, P[L]["tq"], tpe_out[L], l, cap_sp)
+            ca2.ca2_tpe_add(h, g0[0], 0, ptr(tpe_table), P[L]["tq"], ptr(tpe_out[L]), l, cap_sp)
         gt.capture_end()
     gt.replay()
     torch.cuda.synchronize()
@@ -373,17 +408,19 @@ def run_ca2(args):
     # (random weights per block, bias included) stored straight into the ring and spatial
     # cache; 28 launches in a CUDA graph, replayed 5 times.  The queue is full, so 8 frames
     # are evicted first and committed back afterwards (the same queue length as the step).
-    C = H * D
+    # the projection's input rows are the full hidden state (Cin = H_all*D, the row pitch);
+    # its outputs are this process's heads' K and V channels
+    C, Cin = H * D, H_all * D
     n_sp = min(PS, l)
-    wk = [[(torch.randn((2 * C, C), generator=g, device=dev) * C ** -0.5).to(torch.bfloat16) for _ in range(2)]
-          for _ in range(NL)]
+    wk = [[(torch.randn((2 * C, Cin), generator=g, device=dev) * Cin ** -0.5).to(torch.bfloat16)
+           for _ in range(2)] for _ in range(NL)]
     bk = [(torch.randn((2 * C,), generator=g, device=dev) * 0.1).to(torch.bfloat16) for _ in range(NL)]
     cache.evict_for(l)
     gp = torch.cuda.CUDAGraph()
     with torch.cuda.stream(cap):
         gp.capture_begin()
         for L in range(NL):
-            ca2.ca2_kv_proj_write(h, L, P[L]["tk"], wk[L][0], bk[L], P[L]["sk"], wk[L][1], bk[L], l, cap_sp)
+            ca2.ca2_kv_proj_write(h, L, inp[L]["tk"], wk[L][0], bk[L], inp[L]["sk"], wk[L][1], bk[L], l, cap_sp)
         gp.capture_end()
     gp.replay()
     torch.cuda.synchronize()
@@ -404,7 +441,7 @@ def run_ca2(args):
     s_flops_self = 4 * D * HW * HW * l * H * B                     # self-repeat mode (own frame once)
     w_bytes = 2 * NL * (2 * l + 2 * PS) * frame_bytes              # read + write of K,V (temporal, spatial)
     tpe_bytes = 2 * l * frame_bytes + l * H * D * 2                 # chunk read + write, n table rows
-    proj_flops = 2 * B * HW * (l + n_sp) * 2 * C * C               # temporal + spatial [K | V] = x W^T
+    proj_flops = 2 * B * HW * (l + n_sp) * 2 * C * Cin             # temporal + spatial [K | V] = x W^T
     avg_t = statistics.mean(tp_ms) / 1e3
     avg_sd = statistics.mean(sp_den) / 1e3
     avg_ss = statistics.mean(sp_self) / 1e3
@@ -442,16 +479,18 @@ def run_ca2(args):
     # ---- end to end through host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, inp, so, to, step, stream, NL, tokens_per_step, world, dist, add_set, cur)
+        e2e = run_e2e(args, inp, so, to, step, stream, NL, job_tokens, world, dist, add_set, cur, hv)
 
     out = {
         "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+        "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.49) bf16 Q/K/V; no weights needed)",
-        "config": {"workload": cfg["name"], "config": args.config, "batch": B, "tokens_per_frame": HW, "heads": H,
-                   "head_dim": D, "chunk_len": l, "p_max": PM, "p_spatial": PS, "blocks": NL,
-                   "denoise_steps": T, "queue_len": PM, "parallelism": "replica per GPU (dp%d)" % world,
+        "config": {"workload": cfg["name"], "config": args.config, "batch": B, "tokens_per_frame": HW,
+                   "heads": H_all, "head_dim": D, "chunk_len": l, "p_max": PM, "p_spatial": PS, "blocks": NL,
+                   "denoise_steps": T, "queue_len": PM, "parallelism": parallelism(sharded, world, groups, grank,
+                                                                                  h0, H, H_all),
                    "l2": "inputs larger than L2: %d per-block caches and inputs, %.2f GB on the device"
                          % (NL, resident_gb),
                    "tokens_per_step": tokens_per_step},
@@ -471,15 +510,25 @@ def run_ca2(args):
         print(json.dumps(out))
 
 
-def run_e2e(args, inp, so, to, step_fn, stream, NL, tokens_per_step, world, dist, add_set, cur):
+def parallelism(sharded, world, groups, grank, h0, H, H_all):
+    if not sharded:
+        return "replica per GPU (dp%d)" % world
+    if world > 1:
+        return "heads split over %d ranks (tp%d; rank 0 runs heads %d..%d of %d)" % (world, world, h0, h0 + H - 1,
+                                                                                 H_all)
+    return ("one group of a %d-way head split timed alone: heads %d..%d of %d (group %d); value counts its "
+            "heads' share of each token" % (groups, h0, h0 + H - 1, H_all, grank))
+
+
+def run_e2e(args, inp, so, to, step_fn, stream, NL, job_tokens, world, dist, add_set, cur, hv):
     """The same step with its inputs copied from pinned host memory and its outputs read
     back, all inside the timed region.  The copies run on two streams of their own against
     two device sets of inputs and outputs: while step k computes on one set, step k+1's
     inputs are copied into the other, and step k's outputs are read back while step k+1
     computes.  Events order every copy against the steps that use its buffers."""
     import torch
-    host_in = [{k: v.cpu().pin_memory() for k, v in d.items()} for d in inp]
-    host_out = [torch.empty((so if i % 2 == 0 else to)[0].shape, dtype=torch.bfloat16).pin_memory()
+    host_in = [{k: hv(v).contiguous().cpu().pin_memory() for k, v in d.items()} for d in inp]
+    host_out = [torch.empty(hv((so if i % 2 == 0 else to)[0]).shape, dtype=torch.bfloat16).pin_memory()
                 for i in range(2 * NL)]
     h2d = sum(v.numel() * 2 for d in host_in for v in d.values())
     d2h = sum(t.numel() * 2 for t in host_out)
@@ -498,7 +547,7 @@ def run_e2e(args, inp, so, to, step_fn, stream, NL, tokens_per_step, world, dist
                 up.wait_event(ev_comp[i])          # the step that last read this set is done
             for L in range(NL):
                 for key, v in host_in[L].items():
-                    din[L][key].copy_(v, non_blocking=True)
+                    hv(din[L][key]).copy_(v, non_blocking=True)
             ev_h2d[i].record(up)
 
     def compute(k):
@@ -516,8 +565,8 @@ def run_e2e(args, inp, so, to, step_fn, stream, NL, tokens_per_step, world, dist
         with torch.cuda.stream(down):
             down.wait_event(ev_comp[i])
             for L in range(NL):
-                host_out[2 * L].copy_(dso[L], non_blocking=True)
-                host_out[2 * L + 1].copy_(dto[L], non_blocking=True)
+                host_out[2 * L].copy_(hv(dso[L]), non_blocking=True)
+                host_out[2 * L + 1].copy_(hv(dto[L]), non_blocking=True)
             ev_d2h[i].record(down)
 
     def run(n_steps, start=None):
@@ -547,7 +596,7 @@ def run_e2e(args, inp, so, to, step_fn, stream, NL, tokens_per_step, world, dist
     torch.cuda.synchronize()
     cur[0] = 0
     ms = max_over_ranks(a.elapsed_time(b), dist, world, "cuda")
-    return {"value": whole_job_rate(tokens_per_step, steps, world, ms), "unit": "query-tokens/s",
+    return {"value": whole_job_rate(job_tokens, steps, 1, ms), "unit": "query-tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
             "copies": "host<->device copies on two streams of their own, overlapping the steps "

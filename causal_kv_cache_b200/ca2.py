@@ -21,7 +21,7 @@ __all__ = [
     "ca2_cache_config", "ca2_cache_layer_offsets",
     "ca2_cache_write", "ca2_kv_proj_write", "ca2_cache_commit", "ca2_temporal_attn", "ca2_spatial_prefix_attn",
     "ca2_tpe_indices", "ca2_tpe_add",
-    "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string",
+    "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string", "ca2_head_shard",
     "ca2_last_error_string",
     "KVCache", "STATUS",
 ]
@@ -91,6 +91,7 @@ def load_library(path: Optional[str] = None):
         "ca2_cache_state": ([vp, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(ll)], i),
         "ca2_device_status": ([], i),
         "ca2_selftest_timeout": ([i, vp], i),
+        "ca2_head_shard": ([i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)], i),
         "ca2_status_string": ([i], ctypes.c_char_p),
         "ca2_last_error_string": ([], ctypes.c_char_p),
     }
@@ -258,6 +259,14 @@ def ca2_device_status() -> int:
 
 def ca2_selftest_timeout(wait_us: int, stream=None) -> None:
     _check(load_library().ca2_selftest_timeout(int(wait_us), _stream(stream)), "ca2_selftest_timeout")
+
+
+def ca2_head_shard(heads: int, world: int, rank: int) -> Tuple[int, int]:
+    """(first head, number of heads) that `rank` of `world` owns."""
+    h0, hc = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load_library().ca2_head_shard(int(heads), int(world), int(rank), ctypes.byref(h0), ctypes.byref(hc)),
+           "ca2_head_shard")
+    return h0.value, hc.value
 
 
 def ca2_status_string(status: int) -> str:

@@ -530,6 +530,15 @@ int ca2_selftest_timeout(int wait_us, void *stream)
         ca2::launch_timeout_selftest((unsigned long long)wait_us * 1000ull, static_cast<cudaStream_t>(stream)));
 }
 
+int ca2_head_shard(int heads, int world, int rank, int *h0, int *h_count)
+{
+    if (world < 1 || heads < world || rank < 0 || rank >= world) return CA2_ERR_SHAPE;
+    const int base = heads / world, extra = heads % world;
+    if (h0) *h0 = rank * base + (rank < extra ? rank : extra);
+    if (h_count) *h_count = base + (rank < extra ? 1 : 0);
+    return CA2_OK;
+}
+
 const char *ca2_last_error_string(void) { return g_last_cuda_error; }
 
 const char *ca2_status_string(int s)

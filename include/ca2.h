@@ -233,6 +233,14 @@ int ca2_device_status(void);
  * CA2_ERR_TIMEOUT.  1 <= wait_us <= 1000000. */
 int ca2_selftest_timeout(int wait_us, void *stream);
 
+/* Head partition for running one layer on `world` ranks without a collective on the path:
+ * every temporal (token, head) history and every spatial (frame, head) map is independent, so
+ * a rank owns the contiguous heads [*h0, *h0 + *h_count) of every layer (caches sized for
+ * h_count heads) and runs them on the full-width activations through ca2_config.row_pitch.
+ * The first (heads mod world) ranks take one head more.  Host-only.  1 <= world <= heads and
+ * 0 <= rank < world, else CA2_ERR_SHAPE; either out pointer may be NULL. */
+int ca2_head_shard(int heads, int world, int rank, int *h0, int *h_count);
+
 /* Static description of an error code. */
 const char *ca2_status_string(int status);
 

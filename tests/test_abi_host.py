@@ -285,3 +285,22 @@ def test_layer_offsets_follow_the_documented_layout():
         with pytest.raises(ca2.Ca2Error):
             ca2.ca2_cache_layer_offsets(h, *bad)
     ca2.ca2_cache_destroy(h)
+
+
+def test_head_shard_partition():
+    """ca2_head_shard: for every head count up to 32 and every world size up to it, the ranks'
+    ranges are contiguous, in rank order, cover [0, H) once, and differ in size by at most one
+    (the larger ones first); bad arguments are rejected."""
+    for H in range(1, 33):
+        for world in range(1, H + 1):
+            parts = [ca2.ca2_head_shard(H, world, r) for r in range(world)]
+            assert parts[0][0] == 0
+            for (a0, ac), (b0, _) in zip(parts, parts[1:]):
+                assert b0 == a0 + ac
+            assert parts[-1][0] + parts[-1][1] == H
+            sizes = [hc for _, hc in parts]
+            assert min(sizes) >= 1 and max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+    for bad in ((4, 0, 0), (4, 5, 0), (4, 2, 2), (4, 2, -1), (0, 1, 0)):
+        with pytest.raises(ca2.Ca2Error) as e:
+            ca2.ca2_head_shard(*bad)
+        assert e.value.status == -2
