@@ -3,7 +3,8 @@
 // Ca2-VDM ("Ca2-VDM" papernotes page, 整体框架 and 关键设计 4-5): after a chunk is denoised,
 // one clean forward pass computes its K/V, which join the temporal queue (FIFO, at most
 // Pmax frames) and replace the one-chunk spatial cache.  This kernel is the data movement
-// of that step for every layer at once: a bit-exact copy, 16 bytes per access.  The ring
+// of that step for every layer at once: a copy, 16 bytes per access (K bit for bit, V as
+// the exact fp16 form of each bf16 value).  The ring
 // is token-major and head-major within a token ([B][HW][H][Pmax][D]: one head's Pmax slots
 // are contiguous), so a temporal write moves each (token, frame, head) row of D elements of
 // the chunk into that head's slot.
@@ -18,7 +19,7 @@ __device__ int g_status = 0;
 
 namespace {
 constexpr int kThreads = 256;
-constexpr int kVecPerThread = 4;
+constexpr int kUnroll = 4;        // loads in flight per lane
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 {
@@ -31,85 +32,113 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 }  // namespace
 
 // blockIdx.y = (layer, tensor): tensor 0/1 = temporal K/V, 2/3 = spatial K/V.
-//   temporal: chunk [B][HW][n][H][D] -> ring [B][HW][H][Pmax][D]; (token, j, h) -> slot (slot0 + j) mod Pmax
-//   spatial : chunk [B][n][HW][C], its last n_sp frames -> spatial cache [n_sp][B][HW][C]
-//   (K copied, V converted to fp16)
-// (source rows are src_row_vec 16-byte vectors apart, of which the first row_vec are copied)
+// The copy is cut into runs that are contiguous in the destination:
+//   temporal: run (token, h) = head h of the chunk's n rows of that token -> the head's n
+//             consecutive ring slots (slot0 + j) mod Pmax: n * head_vec vectors (two pieces
+//             when the slots wrap past Pmax);
+//   spatial : run (jsp, b, s) = one row of the chunk's frame n - n_sp + jsp -> one row of the
+//             spatial cache [n_sp][B][HW][C].
+// A warp takes whole runs (grid-stride over the runs) and its lanes take a run's vectors in
+// order, 32 at a time, so a warp's stores cover up to 512 contiguous bytes: the ring's
+// 32-byte sectors are written whole except at a run's two ends.  Each lane keeps up to
+// kUnroll loads in flight.  K is copied; V is converted to fp16.  Source rows are
+// src_row_vec 16-byte vectors apart.
 __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams p)
 {
     const int li = blockIdx.y >> 2;
     const int tensor = blockIdx.y & 3;
     const CacheWriteLayer &Ly = p.layer[li];
     const long long layer = p.layer0 + li;
-    const long long rv = p.row_vec;
-    long long total;
-    const uint4 *src;
-    uint4 *dst;
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = ((long long)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const long long n_warps = (long long)gridDim.x * (kThreads / 32);
+    const bool is_v = (tensor & 1) != 0;
+    uint32_t vmax = 0;       // max |v| bits per half, V tensors only
+
+    // V: the fp16 form of each bf16 element (exact within the fp16 range); elements beyond it
+    // (|v| >= 65536, inf, NaN) are recorded as a range error below
+    auto to_f16 = [&](uint4 &x) {
+        vmax = __vmaxu2(vmax, abs_max4(x.x, x.y, x.z, x.w));
+        x = make_uint4(pack_f16x2(bf16_lo(x.x), bf16_hi(x.x)), pack_f16x2(bf16_lo(x.y), bf16_hi(x.y)),
+                       pack_f16x2(bf16_lo(x.z), bf16_hi(x.z)), pack_f16x2(bf16_lo(x.w), bf16_hi(x.w)));
+    };
+
     if (tensor < 2) {
-        total = p.tokens * p.n * rv;
-        src = tensor == 0 ? Ly.kt : Ly.vt;
-        dst = p.tbuf + ((layer * 2 + tensor) * p.tokens) * p.p_max * rv;
-    } else {
-        total = (long long)p.n_sp * p.tokens * rv;
-        src = tensor == 2 ? Ly.ks : Ly.vs;
-        dst = p.sbuf + ((layer * 2 + (tensor - 2)) * p.p_spatial) * p.tokens * rv;
-    }
-    const long long base = (long long)blockIdx.x * (kThreads * kVecPerThread) + threadIdx.x;
-    if (base >= total) return;
-    uint4 v[kVecPerThread];
-    long long so[kVecPerThread], dof[kVecPerThread];
+        const uint4 *src = tensor == 0 ? Ly.kt : Ly.vt;
+        uint4 *dst = p.tbuf + ((layer * 2 + tensor) * p.tokens) * p.p_max * p.row_vec;
+        const int hv = p.head_vec;
+        const int run_len = p.n * hv;
+        const long long runs = p.tokens * p.heads;
+        // (frame, vector) of a run position: this lane's first, and the step of 32 positions
+        const int j_first = lane / hv, dv_first = lane - (lane / hv) * hv;
+        const int dj = 32 / hv, ddv = 32 - (32 / hv) * hv;
+        for (long long r = warp0; r < runs; r += n_warps) {
+            const long long tok = r / p.heads;
+            const int h = (int)(r - tok * p.heads);
+            const uint4 *s = src + tok * p.n * p.src_row_vec + (long long)h * hv;
+            uint4 *d = dst + r * p.p_max * hv;
+            int j = j_first, dv = dv_first;
+            for (int q = lane; q < run_len; q += 32 * kUnroll) {
+                uint4 v[kUnroll];
+                int doff[kUnroll];
 #pragma unroll
-    for (int i = 0; i < kVecPerThread; ++i) {
-        const long long e = base + (long long)i * kThreads;
-        so[i] = dof[i] = -1;
-        if (e < total) {
-            const long long row = e / rv, off = e - row * rv;
-            if (tensor < 2) {
-                const long long tok = row / p.n;
-                const int j = (int)(row - tok * p.n);
-                int slot = p.slot0 + j;
-                if (slot >= p.p_max) slot -= p.p_max;
-                const int h = (int)(off / p.head_vec);
-                const long long dv = off - (long long)h * p.head_vec;
-                so[i] = row * p.src_row_vec + off;
-                dof[i] = ((tok * p.heads + h) * p.p_max + slot) * p.head_vec + dv;
-            } else {
-                // row = jsp * tokens + (b * HW + s); source frame n - n_sp + jsp of video b
-                const long long jsp = row / p.tokens;
-                const long long bt = row - jsp * p.tokens;
-                const long long b = bt / p.hw, sidx = bt - b * p.hw;
-                so[i] = ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * p.src_row_vec + off;
-                dof[i] = e;
+                for (int u = 0; u < kUnroll; ++u) {
+                    doff[u] = -1;
+                    if (q + 32 * u < run_len) {
+                        v[u] = ld_stream(s + (long long)j * p.src_row_vec + dv);
+                        int slot = p.slot0 + j;
+                        if (slot >= p.p_max) slot -= p.p_max;
+                        doff[u] = slot * hv + dv;
+                    }
+                    dv += ddv;
+                    j += dj;
+                    if (dv >= hv) { dv -= hv; ++j; }
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    if (doff[u] < 0) continue;
+                    if (is_v) to_f16(v[u]);
+                    d[doff[u]] = v[u];
+                }
             }
-            v[i] = ld_stream(src + so[i]);
+        }
+    } else {
+        const uint4 *src = tensor == 2 ? Ly.ks : Ly.vs;
+        uint4 *dst = p.sbuf + ((layer * 2 + (tensor - 2)) * p.p_spatial) * p.tokens * p.row_vec;
+        const int rv = (int)p.row_vec;
+        const long long runs = (long long)p.n_sp * p.tokens;
+        for (long long r = warp0; r < runs; r += n_warps) {
+            // r = jsp * tokens + (b * HW + s): source frame n - n_sp + jsp of video b
+            const long long jsp = r / p.tokens;
+            const long long bt = r - jsp * p.tokens;
+            const long long b = bt / p.hw, sidx = bt - b * p.hw;
+            const uint4 *s = src + ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * p.src_row_vec;
+            uint4 *d = dst + r * rv;
+            for (int q = lane; q < rv; q += 32 * kUnroll) {
+                uint4 v[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    if (q + 32 * u < rv) v[u] = ld_stream(s + q + 32 * u);
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    if (q + 32 * u >= rv) continue;
+                    if (is_v) to_f16(v[u]);
+                    d[q + 32 * u] = v[u];
+                }
+            }
         }
     }
-    if (tensor & 1) {
-        // both caches keep V in fp16, the operand type of the attention's P V products: the
-        // exact value of each bf16 element within the fp16 range; elements beyond it
-        // (|v| >= 65536, inf, NaN) are recorded as a range error
-        uint32_t vmax = 0;
-#pragma unroll
-        for (int i = 0; i < kVecPerThread; ++i) {
-            if (dof[i] < 0) continue;
-            vmax = __vmaxu2(vmax, abs_max4(v[i].x, v[i].y, v[i].z, v[i].w));
-            v[i] = make_uint4(pack_f16x2(bf16_lo(v[i].x), bf16_hi(v[i].x)), pack_f16x2(bf16_lo(v[i].y), bf16_hi(v[i].y)),
-                              pack_f16x2(bf16_lo(v[i].z), bf16_hi(v[i].z)), pack_f16x2(bf16_lo(v[i].w), bf16_hi(v[i].w)));
-        }
-        if ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u) record_status(kStatusRange);
-    }
-#pragma unroll
-    for (int i = 0; i < kVecPerThread; ++i)
-        if (dof[i] >= 0) dst[dof[i]] = v[i];
+    if (is_v && ((vmax & 0xFFFFu) >= 0x4780u || (vmax >> 16) >= 0x4780u)) record_status(kStatusRange);
 }
 
 cudaError_t launch_cache_write(const CacheWriteParams &p, cudaStream_t stream)
 {
-    const long long per_block = (long long)kThreads * kVecPerThread;
-    const long long t_total = p.tokens * p.n * p.row_vec;
-    const long long s_total = (long long)p.n_sp * p.tokens * p.row_vec;
-    const long long most = t_total > s_total ? t_total : s_total;
-    dim3 grid((unsigned)((most + per_block - 1) / per_block), (unsigned)(p.n_layers * 4));
+    // about two temporal runs per warp; the spatial blocks of the same grid stride over fewer
+    const long long t_runs = p.tokens * p.heads;
+    const long long s_runs = (long long)p.n_sp * p.tokens;
+    const long long warps = (t_runs + 1) / 2 > s_runs ? (t_runs + 1) / 2 : s_runs;
+    const long long gx = (warps + kThreads / 32 - 1) / (kThreads / 32);
+    dim3 grid((unsigned)(gx < 65535 ? gx : 65535), (unsigned)(p.n_layers * 4));
     if (grid.x == 0 || grid.y == 0) return cudaSuccess;
     // a plain launch: it starts only after the previous kernel on the stream (the last
     // attention pass reads the cache) has completed
