@@ -22,6 +22,7 @@ __all__ = [
     "ca2_cache_write", "ca2_kv_proj_write", "ca2_cache_commit", "ca2_temporal_attn", "ca2_spatial_prefix_attn",
     "ca2_tpe_indices", "ca2_tpe_add",
     "ca2_cache_state", "ca2_device_status", "ca2_selftest_timeout", "ca2_status_string", "ca2_head_shard",
+    "ca2_debug_build",
     "ca2_last_error_string",
     "KVCache", "STATUS",
 ]
@@ -31,6 +32,7 @@ LIBRARY_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libca2.
 STATUS = {
     0: "CA2_OK", -1: "CA2_ERR_ARG", -2: "CA2_ERR_SHAPE", -3: "CA2_ERR_CAPACITY",
     -4: "CA2_ERR_ALIGN", -5: "CA2_ERR_CUDA", -6: "CA2_ERR_TIMEOUT", -7: "CA2_ERR_RANGE",
+    -8: "CA2_ERR_BOUNDS",
 }
 
 
@@ -92,6 +94,7 @@ def load_library(path: Optional[str] = None):
         "ca2_device_status": ([], i),
         "ca2_selftest_timeout": ([i, vp], i),
         "ca2_head_shard": ([i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)], i),
+        "ca2_debug_build": ([], i),
         "ca2_status_string": ([i], ctypes.c_char_p),
         "ca2_last_error_string": ([], ctypes.c_char_p),
     }
@@ -267,6 +270,11 @@ def ca2_head_shard(heads: int, world: int, rank: int) -> Tuple[int, int]:
     _check(load_library().ca2_head_shard(int(heads), int(world), int(rank), ctypes.byref(h0), ctypes.byref(hc)),
            "ca2_head_shard")
     return h0.value, hc.value
+
+
+def ca2_debug_build() -> bool:
+    """True when the loaded library is the bounds-checked debug build."""
+    return bool(load_library().ca2_debug_build())
 
 
 def ca2_status_string(status: int) -> str:

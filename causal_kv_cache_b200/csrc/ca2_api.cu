@@ -287,6 +287,11 @@ int ca2_cache_write(ca2_cache *c, const void *const *k_t, const void *const *v_t
     p.p_max = g.p_max;
     p.n_sp = n_sp;
     p.p_spatial = g.p_spatial;
+    // extents for the debug build's bounds checks
+    p.t_src_vec = (p.tokens * n - 1) * p.src_row_vec + p.row_vec;
+    p.s_src_vec = ((long long)g.batch * n * g.hw - 1) * p.src_row_vec + p.row_vec;
+    p.tbuf_vec = (long long)g.n_layers * 2 * p.tokens * g.p_max * p.row_vec;
+    p.sbuf_vec = (long long)g.n_layers * 2 * g.p_spatial * p.tokens * p.row_vec;
     for (int L0 = 0; L0 < g.n_layers; L0 += ca2::kMaxLayersPerWrite) {
         const int nl = (g.n_layers - L0) < ca2::kMaxLayersPerWrite ? (g.n_layers - L0) : ca2::kMaxLayersPerWrite;
         p.layer0 = L0;
@@ -329,6 +334,8 @@ int ca2_temporal_attn(ca2_cache *c, int layer, const void *q, const void *k, con
     p.ring_box_mask = 0;
     for (int i = 0; i < c->count; ++i) p.ring_box_mask |= 1u << (((c->head + i) % g.p_max) / 16);
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)g.head_dim));
+    p.ring_bytes = (long long)g.batch * g.hw * g.heads * g.p_max * g.head_dim * 2;
+    p.out_elems = ((long long)g.batch * g.hw * n - 1) * g.row_pitch + (long long)g.heads * g.head_dim;
 
     // temporal chunk tensors are token-major [B][HW][n][H][D] (C = H*D), read as TMA boxes;
     // the ring [B][HW][H][Pmax][D] is read with bulk copies of one head's consecutive slots
@@ -436,6 +443,8 @@ int ca2_kv_proj_write(ca2_cache *c, int layer, const void *x_t, const void *w_t,
     const long long tiles_s = (long long)g.batch * n_sp * p.tiles_s_frame * p.tiles_n;
     if (p.tiles_t + tiles_s >= (1ll << 31)) return CA2_ERR_SHAPE;
     p.total_tiles = (int)(p.tiles_t + tiles_s);
+    p.ring_elems = (long long)g.batch * g.hw * g.heads * g.p_max * g.head_dim;
+    p.sp_elems = (long long)g.p_spatial * g.batch * g.hw * g.heads * g.head_dim;
 
     // x_t: [B*HW*n][Cin]; x_s: (Cin, HW, B*n frames); W: [2C][Cin] (output channel rows)
     ca2::KvProjMaps m;
@@ -491,6 +500,8 @@ int ca2_tpe_add(const ca2_cache *c, long long first_global_frame, int offset, co
     if (p.rows * p.pitch_vec >= (1ll << 31) || (long long)n_tpe * p.pitch_vec >= (1ll << 31)) return CA2_ERR_SHAPE;
     for (int i = 0; i < ca2::kMaxChunk; ++i)
         p.tpe_row[i] = i < n ? (int)(((long long)offset + first_global_frame + i) % n_tpe) : 0;
+    p.xo_vec = (p.rows - 1) * p.pitch_vec + p.row_vec;
+    p.table_vec = (n_tpe - 1) * p.pitch_vec + p.row_vec;
     return cuda_status(ca2::launch_tpe_add(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -520,6 +531,7 @@ int ca2_device_status(void)
     int s = 0;
     if (ca2::read_and_clear_status(&s) != 0) return CA2_ERR_CUDA;
     if (s == 0) return CA2_OK;
+    if (s >= ca2::kStatusBoundsCode) return CA2_ERR_BOUNDS;
     return s >= ca2::kStatusRangeCode ? CA2_ERR_RANGE : CA2_ERR_TIMEOUT;
 }
 
@@ -539,6 +551,15 @@ int ca2_head_shard(int heads, int world, int rank, int *h0, int *h_count)
     return CA2_OK;
 }
 
+int ca2_debug_build(void)
+{
+#ifdef CA2_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 const char *ca2_last_error_string(void) { return g_last_cuda_error; }
 
 const char *ca2_status_string(int s)
@@ -552,6 +573,7 @@ const char *ca2_status_string(int s)
     case CA2_ERR_CUDA: return "CUDA runtime error";
     case CA2_ERR_TIMEOUT: return "device wait timed out";
     case CA2_ERR_RANGE: return "input value outside the supported range";
+    case CA2_ERR_BOUNDS: return "bounds check failed (debug build)";
     default: return "unknown status";
     }
 }

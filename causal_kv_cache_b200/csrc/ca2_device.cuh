@@ -38,6 +38,20 @@ __device__ __forceinline__ void record_status(int code)
     atomicCAS(&g_status, 0, code);
 }
 
+// Bounds checks of the debug build (compiled with -DCA2_DEBUG, libca2_debug.so): every
+// global access a kernel addresses itself (plain loads and stores, bulk copies) is checked
+// against the extent of its buffer.  A failed check records kStatusBounds + site and the
+// access is skipped; nothing traps.  Release builds compile the checks out (the condition is
+// not evaluated).  Accesses through tensor maps are bounded by the maps' extents, which the
+// TMA unit enforces in both builds.  (The same value as kStatusBoundsCode on the host side.)
+constexpr int kStatusBounds = 2000;
+#ifdef CA2_DEBUG
+#define CA2_IN_BOUNDS(cond, site) \
+    ((cond) ? true : (::ca2::record_status(::ca2::kStatusBounds + (site)), false))
+#else
+#define CA2_IN_BOUNDS(cond, site) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -66,6 +66,8 @@ struct TemporalParams {
     int n_items;    // B * HW * (H / G)
     uint32_t ring_box_mask;   // bit i: ring slots [16i, 16i+16) hold at least one queued frame
     float scale_log2;         // log2(e) / sqrt(D)
+    long long ring_bytes;     // bytes of one layer's K (or V) ring, from rk (rv)
+    long long out_elems;      // elements of out the call may write, from out
 };
 
 // 5-D views (head dim, frame, head, token, video) of the chunk tensors; boxes of
@@ -103,6 +105,10 @@ struct CacheWriteParams {
     int p_max;
     int n_sp;               // spatial frames written: min(P', n)
     int p_spatial;
+    long long t_src_vec;    // 16-byte vectors a temporal source may be read at, from its pointer
+    long long s_src_vec;    // the same for a spatial source
+    long long tbuf_vec;     // 16-byte vectors of the whole temporal buffer, from tbuf
+    long long sbuf_vec;     // the same for the spatial buffer
 };
 
 cudaError_t launch_cache_write(const CacheWriteParams &p, cudaStream_t stream);
@@ -135,6 +141,8 @@ struct TpeAddParams {
     int pitch_vec;          // 16-byte vectors from one row of x, out or table to the next
     int n;                  // chunk frames
     int tpe_row[kMaxChunk]; // table row of each chunk frame
+    long long xo_vec;       // 16-byte vectors of x (and of out) the call may touch
+    long long table_vec;    // 16-byte vectors of the table
 };
 
 cudaError_t launch_tpe_add(const TpeAddParams &p, cudaStream_t stream);
@@ -163,6 +171,8 @@ struct KvProjParams {
     int tiles_s_frame;      // spatial row tiles per frame: ceil(HW / 128)
     int k_steps;            // ceil(C / 64)
     int total_tiles;        // temporal + spatial tiles (the persistent grid walks them)
+    long long ring_elems;   // elements of one layer's K (or V) ring, from ring_k (ring_v)
+    long long sp_elems;     // elements of one layer's spatial K (or V), from sp_k (sp_v)
 };
 
 // A tiles: boxes of 64 channels x 128 rows (x 1 frame); W tiles: 64 channels x kProjBN rows;
@@ -178,6 +188,8 @@ cudaError_t launch_kv_proj(const KvProjMaps &maps, const KvProjParams &p, int gr
 // 0 = fine; codes below kStatusRangeCode name the bounded wait that gave up, codes from it on
 // an input value outside the supported range (device code records them with record_status).
 constexpr int kStatusRangeCode = 1000;
+// codes from kStatusBoundsCode on: a failed bounds check of the debug build (site added)
+constexpr int kStatusBoundsCode = 2000;
 
 // ---- bounded-wait self test ---------------------------------------------------------------
 cudaError_t launch_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);

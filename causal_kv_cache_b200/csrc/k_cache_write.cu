@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
 
     if (tensor < 2) {
         const uint4 *src = tensor == 0 ? Ly.kt : Ly.vt;
-        uint4 *dst = p.tbuf + ((layer * 2 + tensor) * p.tokens) * p.p_max * p.row_vec;
+        const long long dst0 = ((layer * 2 + tensor) * p.tokens) * p.p_max * p.row_vec;
+        uint4 *dst = p.tbuf + dst0;
         const int hv = p.head_vec;
         const int run_len = p.n * hv;
         const long long runs = p.tokens * p.heads;
@@ -75,8 +76,10 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
         for (long long r = warp0; r < runs; r += n_warps) {
             const long long tok = r / p.heads;
             const int h = (int)(r - tok * p.heads);
-            const uint4 *s = src + tok * p.n * p.src_row_vec + (long long)h * hv;
-            uint4 *d = dst + r * p.p_max * hv;
+            const long long s0 = tok * p.n * p.src_row_vec + (long long)h * hv;
+            const long long d0 = r * p.p_max * hv;
+            const uint4 *s = src + s0;
+            uint4 *d = dst + d0;
             int j = j_first, dv = dv_first;
             for (int q = lane; q < run_len; q += 32 * kUnroll) {
                 uint4 v[kUnroll];
@@ -85,10 +88,12 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
                 for (int u = 0; u < kUnroll; ++u) {
                     doff[u] = -1;
                     if (q + 32 * u < run_len) {
-                        v[u] = ld_stream(s + (long long)j * p.src_row_vec + dv);
+                        const long long so = (long long)j * p.src_row_vec + dv;
+                        v[u] = CA2_IN_BOUNDS(s0 + so < p.t_src_vec, 21) ? ld_stream(s + so) : make_uint4(0u, 0u, 0u, 0u);
                         int slot = p.slot0 + j;
                         if (slot >= p.p_max) slot -= p.p_max;
                         doff[u] = slot * hv + dv;
+                        if (!CA2_IN_BOUNDS(dst0 + d0 + doff[u] < p.tbuf_vec, 22)) doff[u] = -1;
                     }
                     dv += ddv;
                     j += dj;
@@ -104,7 +109,8 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
         }
     } else {
         const uint4 *src = tensor == 2 ? Ly.ks : Ly.vs;
-        uint4 *dst = p.sbuf + ((layer * 2 + (tensor - 2)) * p.p_spatial) * p.tokens * p.row_vec;
+        const long long dst0 = ((layer * 2 + (tensor - 2)) * p.p_spatial) * p.tokens * p.row_vec;
+        uint4 *dst = p.sbuf + dst0;
         const int rv = (int)p.row_vec;
         const long long runs = (long long)p.n_sp * p.tokens;
         for (long long r = warp0; r < runs; r += n_warps) {
@@ -112,16 +118,20 @@ __global__ void __launch_bounds__(kThreads) k_cache_write(const CacheWriteParams
             const long long jsp = r / p.tokens;
             const long long bt = r - jsp * p.tokens;
             const long long b = bt / p.hw, sidx = bt - b * p.hw;
-            const uint4 *s = src + ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * p.src_row_vec;
+            const long long s0 = ((b * p.n + (p.n - p.n_sp + jsp)) * p.hw + sidx) * p.src_row_vec;
+            const uint4 *s = src + s0;
             uint4 *d = dst + r * rv;
             for (int q = lane; q < rv; q += 32 * kUnroll) {
                 uint4 v[kUnroll];
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u)
-                    if (q + 32 * u < rv) v[u] = ld_stream(s + q + 32 * u);
+                    if (q + 32 * u < rv)
+                        v[u] = CA2_IN_BOUNDS(s0 + q + 32 * u < p.s_src_vec, 23) ? ld_stream(s + q + 32 * u)
+                                                                               : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u) {
                     if (q + 32 * u >= rv) continue;
+                    if (!CA2_IN_BOUNDS(dst0 + r * rv + q + 32 * u < p.sbuf_vec, 24)) continue;
                     if (is_v) to_f16(v[u]);
                     d[q + 32 * u] = v[u];
                 }

@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
                     const int h = rem / p.D;
                     const int dd = rem - h * p.D;
                     float b8[8];
-                    bias8(bias, ch, b8);
+                    bias8(CA2_IN_BOUNDS(ch + 8 <= 2 * p.C, 42) ? bias : nullptr, ch, b8);
                     uint4 w;
                     w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) + b8[0], __uint_as_float(v[8 * q + 1]) + b8[1]);
                     w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + b8[2], __uint_as_float(v[8 * q + 3]) + b8[3]);
@@ -268,8 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_kv_proj(const __grid_constant__
                         w = make_uint4(pack_f16x2(bf16_lo(w.x), bf16_hi(w.x)), pack_f16x2(bf16_lo(w.y), bf16_hi(w.y)),
                                        pack_f16x2(bf16_lo(w.z), bf16_hi(w.z)), pack_f16x2(bf16_lo(w.w), bf16_hi(w.w)));
                     }
-                    __nv_bfloat16 *dst = (kv ? dst_v : dst_k) + base + (long long)h * head_stride + dd;
-                    *reinterpret_cast<uint4 *>(dst) = w;
+                    const long long off = base + (long long)h * head_stride + dd;
+                    if (CA2_IN_BOUNDS(off + 8 <= (d.spatial ? p.sp_elems : p.ring_elems), 41))
+                        *reinterpret_cast<uint4 *>((kv ? dst_v : dst_k) + off) = w;
                 }
             }
             // the accumulator may take the tile after next

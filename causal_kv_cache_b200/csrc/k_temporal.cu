@@ -271,8 +271,11 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
                         const int kv = lane / G;
                         const size_t off = ((((size_t)b * p.HW + (size_t)s) * (size_t)p.H + (size_t)(hg * G + w)) *
                                                 (size_t)p.Pmax + (size_t)s0) * ((size_t)D * 2u);
-                        bulk_g2s(dst + (uint32_t)kv * L.kv_box + (uint32_t)(w * kKeys * D * 2),
-                                 (kv ? p.rv : p.rk) + off, run, full_bar(slot));
+                        // (a skipped copy leaves the stage's barrier short: the consumers' bounded
+                        // wait then gives up, after the bounds record)
+                        if (CA2_IN_BOUNDS(off + run <= (size_t)p.ring_bytes, 11))
+                            bulk_g2s(dst + (uint32_t)kv * L.kv_box + (uint32_t)(w * kKeys * D * 2),
+                                     (kv ? p.rv : p.rk) + off, run, full_bar(slot));
                     }
                 }
             }
@@ -504,15 +507,18 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
             }
             const float i0 = 1.f / l0, i1 = 1.f / l1;
             const int qrow = lane >> 2;
-            __nv_bfloat16 *orow = p.out + (((long long)b * p.HW + s) * p.n + qrow) * p.pitch +
-                                  (long long)(hg * G + w) * D + 2 * (lane & 3);
+            const long long o0 = (((long long)b * p.HW + s) * p.n + qrow) * p.pitch +
+                                 (long long)(hg * G + w) * D + 2 * (lane & 3);
+            __nv_bfloat16 *orow = p.out + o0;
 #pragma unroll
             for (int t = 0; t < DT; ++t) {
                 const uint32_t y0 = movm_t(pack_bf16x2(acc[t][0] * i0, acc[t][1] * i1));
-                if (qrow < p.n) *reinterpret_cast<uint32_t *>(orow + 16 * t) = y0;
+                if (qrow < p.n && CA2_IN_BOUNDS(o0 + 16 * t + 2 <= p.out_elems, 12))
+                    *reinterpret_cast<uint32_t *>(orow + 16 * t) = y0;
                 if (16 * t + 16 <= D) {
                     const uint32_t y1 = movm_t(pack_bf16x2(acc[t][2] * i0, acc[t][3] * i1));
-                    if (qrow < p.n) *reinterpret_cast<uint32_t *>(orow + 16 * t + 8) = y1;
+                    if (qrow < p.n && CA2_IN_BOUNDS(o0 + 16 * t + 10 <= p.out_elems, 13))
+                        *reinterpret_cast<uint32_t *>(orow + 16 * t + 8) = y1;
                 }
             }
         }

@@ -50,14 +50,15 @@ __global__ void __launch_bounds__(kThreads) k_tpe_add(const TpeAddParams p)
             const uint32_t v = e - row * rv;                // 16-byte vector within the row
             const uint32_t f = row % n;                     // chunk frame (token-major rows)
             xi[i] = row * pv + v;
-            xv[i] = p.x[xi[i]];
-            tv[i] = p.table[(uint32_t)p.tpe_row[f] * pv + v];
+            const uint32_t ti = (uint32_t)p.tpe_row[f] * pv + v;
+            xv[i] = CA2_IN_BOUNDS(xi[i] < p.xo_vec, 51) ? p.x[xi[i]] : make_uint4(0u, 0u, 0u, 0u);
+            tv[i] = CA2_IN_BOUNDS(ti < p.table_vec, 52) ? p.table[ti] : make_uint4(0u, 0u, 0u, 0u);
         }
     }
 #pragma unroll
     for (int i = 0; i < kVecPerThread; ++i) {
         const uint32_t e = base + (uint32_t)(i * kThreads);
-        if (e < total) p.out[xi[i]] = add8(xv[i], tv[i]);
+        if (e < total && CA2_IN_BOUNDS(xi[i] < p.xo_vec, 53)) p.out[xi[i]] = add8(xv[i], tv[i]);
     }
 }
 

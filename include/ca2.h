@@ -83,8 +83,10 @@ typedef enum {
     CA2_ERR_ALIGN = -4,     /* a pointer is not 16-byte aligned                           */
     CA2_ERR_CUDA = -5,      /* a CUDA runtime call or kernel launch failed                */
     CA2_ERR_TIMEOUT = -6,   /* a kernel's bounded wait gave up (see ca2_device_status)     */
-    CA2_ERR_RANGE = -7      /* a device input outside the supported range (see
+    CA2_ERR_RANGE = -7,     /* a device input outside the supported range (see
                                ca2_device_status): spatial attention takes |V| <= 65504    */
+    CA2_ERR_BOUNDS = -8     /* debug build only: a kernel's bounds check failed and the
+                               access was skipped (see ca2_device_status, ca2_debug_build) */
 } ca2_status;
 
 /* Sizes in bytes of the temporal and spatial cache buffers for a configuration:
@@ -223,8 +225,9 @@ int ca2_cache_state(const ca2_cache *cache, int *head, int *count, int *sp_count
 
 /* Synchronise the current device and return what the kernels of this library recorded since
  * the last call (clearing the record): CA2_ERR_TIMEOUT if a bounded wait gave up,
- * CA2_ERR_RANGE if an input was outside the supported range (the first record wins), else
- * CA2_OK (or CA2_ERR_CUDA if the synchronisation itself fails). */
+ * CA2_ERR_RANGE if an input was outside the supported range, CA2_ERR_BOUNDS if a bounds check
+ * of the debug build failed (the first record wins), else CA2_OK (or CA2_ERR_CUDA if the
+ * synchronisation itself fails). */
 int ca2_device_status(void);
 
 /* Self-test of the bounded-wait path: launches one block that waits on a barrier nothing
@@ -240,6 +243,15 @@ int ca2_selftest_timeout(int wait_us, void *stream);
  * The first (heads mod world) ranks take one head more.  Host-only.  1 <= world <= heads and
  * 0 <= rank < world, else CA2_ERR_SHAPE; either out pointer may be NULL. */
 int ca2_head_shard(int heads, int world, int rank, int *h0, int *h_count);
+
+/* 1 for the debug build (libca2_debug.so, compiled with -DCA2_DEBUG), else 0.  In the debug
+ * build every global access a kernel addresses itself -- plain loads and stores and bulk
+ * copies -- is checked against the extent of its buffer as the call describes it (the
+ * chunk tensors from their pointers and row pitch, the caches from the handle's sizes); a
+ * failed check skips the access and records CA2_ERR_BOUNDS for ca2_device_status.  Accesses
+ * through tensor maps are bounded by the maps in both builds.  The checks cost time; the
+ * release build has none.  Host-only. */
+int ca2_debug_build(void);
 
 /* Static description of an error code. */
 const char *ca2_status_string(int status);

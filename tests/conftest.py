@@ -26,6 +26,20 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
+@pytest.fixture(autouse=True)
+def _device_status_clean(request):
+    """Every GPU test leaves the device status word clear: a timeout, a range error or (in the
+    debug build) a failed bounds check that a test did not read and expect fails the test."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    mod = sys.modules.get("causal_kv_cache_b200.ca2")
+    if mod is None or mod._lib is None:
+        return
+    st = mod.ca2_device_status()
+    assert st == 0, "device status %d (%s) left after the test" % (st, mod.STATUS.get(st, "?"))
+
+
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
     """Raw parity figures of every attention output checked in this session, per workload."""
     mod = sys.modules.get("tests.gpu_util")

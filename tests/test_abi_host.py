@@ -169,7 +169,7 @@ def test_tpe_indices_match_oracle():
 
 
 def test_status_strings():
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         assert ca2.ca2_status_string(code) != "unknown status"
     assert ca2.ca2_status_string(-99) == "unknown status"
 
