@@ -302,6 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
     // of every V tile is set to 1.0 so that the tensor core also accumulates the row sum
     // of the (bf16) probabilities into O[:, D], rescaled together with O.
     const bool ones_col = (p.D & 31) != 0;
+    // columns the P V product actually needs: the head dims plus the ones column, rounded up
+    // to the MMA's N granule of 16 (80 of the 96 loaded at D = 72); the rest stay unused
+    const int dpv = ((p.D + (ones_col ? 1 : 0) + 15) & ~15) < DP ? ((p.D + (ones_col ? 1 : 0) + 15) & ~15) : DP;
 
     if (warp == 0) {
         // ------------------------------- TMA producer (one warp) ----------------------
@@ -344,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
         const int X = warp - 1;
         const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
         constexpr uint32_t idesc_qk = idesc_bf16(kRows, kKeys, false, false);
-        constexpr uint32_t idesc_pv = idesc_f16(kRows, DP, false, true);    // P and V both fp16
+        const uint32_t idesc_pv = idesc_f16(kRows, dpv, false, true);       // P and V both fp16
         // Descriptors are built once; a k-step only adds its byte offset / 16 to the
         // start-address field (addresses stay below 256 KB, so no carry leaves it).
         // K-major (Q, K): 8-row groups 512 B apart; k-step kk = box kk/2, +32 B for odd kk.
@@ -539,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < DP / 16; ++c) {
+                    if (16 * c >= dpv) break;
                     uint32_t o[16];
                     const uint32_t a = o_col + (uint32_t)(16 * c);
                     tmem_ld16(a, o);
@@ -627,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             uint8_t *orow = sgen + L.q0 + X * TB + (size_t)row * (size_t)(p.D * 2);
 #pragma unroll
             for (int c = 0; c < DP / 16; ++c) {
+                if (16 * c >= dpv) break;
                 uint32_t o[16];
                 tmem_ld16(o_col + (uint32_t)(16 * c), o);
 #pragma unroll
