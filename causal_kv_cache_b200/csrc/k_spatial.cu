@@ -451,19 +451,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             const uint32_t vt = sb + L.v0 + s * TB;
             // block jv comes from the own frame when its source index is 0 (see kv_src)
             const bool own = p.n_src == 1 || (jv / p.nkb + 1) % p.n_src == 0;
-            for (int r = lane; own && r < kKeys; r += 32) {
-                const uint32_t rbase = vt + (uint32_t)r * 64u;
-                const uint32_t swz = (uint32_t)((r >> 1) & 3);
-                for (int q = 0; q < pieces; ++q) {
-                    const uint32_t a = rbase + (uint32_t)(q >> 2) * 8192u + ((((uint32_t)q & 3u) ^ swz) << 4);
-                    uint32_t w[4];
-                    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
-                    vmax = __vmaxu2(vmax, abs_max4(w[0], w[1], w[2], w[3]));
+            // 12 pieces in flight per lane: pieces q0..q0+2 of the lane's four rows
+            static_assert(kKeys == 4 * 32, "four rows per lane");
+            for (int q0 = 0; own && q0 < pieces; q0 += 3) {
+                uint32_t w[3][4][4];
+                uint32_t adr[3][4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) w[i] = pack_f16x2(bf16_lo(w[i]), bf16_hi(w[i]));
-                    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                                 : "memory");
-                }
+                for (int dq = 0; dq < 3; ++dq)
+#pragma unroll
+                    for (int ri = 0; ri < 4; ++ri) {
+                        const int q = q0 + dq, r = lane + 32 * ri;
+                        adr[dq][ri] = vt + (uint32_t)r * 64u + (uint32_t)(q >> 2) * 8192u +
+                                      ((((uint32_t)q & 3u) ^ (uint32_t)((r >> 1) & 3)) << 4);
+                        if (q < pieces)
+                            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                                         : "=r"(w[dq][ri][0]), "=r"(w[dq][ri][1]), "=r"(w[dq][ri][2]), "=r"(w[dq][ri][3])
+                                         : "r"(adr[dq][ri]));
+                    }
+#pragma unroll
+                for (int dq = 0; dq < 3; ++dq)
+#pragma unroll
+                    for (int ri = 0; ri < 4; ++ri) {
+                        if (q0 + dq >= pieces) continue;
+                        uint32_t *x = w[dq][ri];
+                        vmax = __vmaxu2(vmax, abs_max4(x[0], x[1], x[2], x[3]));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i] = pack_f16x2(bf16_lo(x[i]), bf16_hi(x[i]));
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(adr[dq][ri]), "r"(x[0]), "r"(x[1]),
+                                     "r"(x[2]), "r"(x[3])
+                                     : "memory");
+                    }
             }
             if (ones_col) {
                 const int c = (D & 31) >> 3;
