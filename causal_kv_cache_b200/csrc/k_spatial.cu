@@ -177,7 +177,7 @@ enum : int {
     B_SFREE = 18,     // 2 [X]: every softmax warp of the tile has read the scores (4 warps)
     B_PFULL = 20,     // 8 [X][c]: probabilities written (4 warps): per chunk in TMEM, or the
                       //           whole block in shared memory ([X][0] only)
-    B_PFREE = 28,     // 2 [X]: the P V product reading P_X in shared memory is done
+    B_UNUSED = 28,    // 2 (free)
     B_ODONE = 30,     // 2 [X]: P V of the block done (all prior products of the tile)
     B_FIN = 32,       // 2 [X]: every product the tile's issuer launched is done
     B_QFULLB = 34,    // Q of tile B
@@ -257,7 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
             mbar_init(bar(B_FIN + i), 1);
         }
         for (int i = 0; i < 2 * kChunks; ++i) mbar_init(bar(B_PFULL + i), 4);
-        for (int i = 0; i < 2; ++i) mbar_init(bar(B_PFREE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm.q);
@@ -408,7 +407,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 if (okc) {
                     tc_fence_after();
                     for (int c = 0; c < kChunks; ++c) issue_pv(j, c);
-                    tc_commit_w(bar(B_PFREE + X));
                 }
             } else {
                 for (int c = 0; c < kChunks; ++c) {
@@ -594,8 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_spatial_prefix(const __grid_con
                 l_sum += ls;
                 if constexpr (kPSmem) {
                     // keys 32c.. -> box c of P_X; this tile's P V of the previous block must be
-                    // done reading P_X before its first chunk is overwritten
-                    if (c == 0 && j > 0 && !warp_wait(bar(B_PFREE + X), (j - 1) & 1, 229, abort_flag)) {
+                    // done reading P_X before its first chunk is overwritten (the block's
+                    // completion barrier, which the rescale above also waits on)
+                    if (c == 0 && j > 0 && !warp_wait(bar(B_ODONE + X), (j - 1) & 1, 229, abort_flag)) {
                         ok = false;
                         break;
                     }
