@@ -168,6 +168,14 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// Hint: bring `bytes` of global memory into L2 (16-byte aligned address and size).  A
+// prefetch only moves data into L2, the point of coherence, so it may run before the
+// previous kernel's writes are complete: later loads still see the current values.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 1-D bulk copy shared -> global (bulk-group completion).
 __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes)
 {

@@ -60,6 +60,8 @@ constexpr int kStages = 4;       // K+V stages in flight per CTA
 constexpr int kKeys = 16;        // key frames per stage
 constexpr int kQ = 8;            // queries per (token, head): the mma N extent
 constexpr float kLazy = 8.0f;    // log2 units
+constexpr int kPrefetchCtas = 128;   // CTAs that prefetch ring runs into L2 before the dependency wait
+constexpr int kPrefetchItems = 4;    // consecutive items each of them covers
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
@@ -196,11 +198,41 @@ __global__ void __launch_bounds__(32 * (kMaxTemporalGroup + 1))
         prefetch_tmap(&tm_v);
     }
     __syncthreads();
+    const int groups = p.H / G;
+    // Before waiting for the previous kernel, the first kPrefetchCtas CTAs (the first
+    // launched, so the ones that start while the previous kernel still runs) ask L2 for the
+    // ring runs of the items the first wave will take: kPrefetchItems consecutive items each.
+    // The ring is cache state, and a prefetch only moves data into L2, so this is safe
+    // whatever the previous kernel writes; the copies after the wait then read L2 instead of
+    // HBM while the previous kernel, if it is compute-bound, leaves HBM idle.
+    if (warp == G && (int)blockIdx.x < kPrefetchCtas && p.ring_box_mask) {
+        const int n_ring_runs = __popc(p.ring_box_mask) * 2 * G;     // (group, tensor, head) runs
+        const int first = (int)blockIdx.x * kPrefetchItems;
+        for (int t = lane; t < kPrefetchItems * n_ring_runs; t += 32) {
+            const int it = first + t / n_ring_runs;
+            if (it >= p.n_items) break;
+            int r = t % n_ring_runs;
+            const int w = r % G;
+            const int kv = (r / G) & 1;
+            int k = r / (2 * G);                                 // k-th set bit of the mask
+            uint32_t mask = p.ring_box_mask;
+            for (; k > 0; --k) mask &= mask - 1;
+            const int box = __ffs(mask) - 1;
+            const int hg = it % groups;
+            const int s = (it / groups) % p.HW;
+            const int b = it / (groups * p.HW);
+            const int s0 = box * kKeys;
+            const int ns = min(kKeys, p.Pmax - s0);
+            const size_t off = ((((size_t)b * p.HW + (size_t)s) * (size_t)p.H + (size_t)(hg * G + w)) *
+                                    (size_t)p.Pmax + (size_t)s0) * ((size_t)D * 2u);
+            if (CA2_IN_BOUNDS(off + (size_t)ns * D * 2 <= (size_t)p.ring_bytes, 14))
+                bulk_prefetch_l2((kv ? p.rv : p.rk) + off, (uint32_t)(ns * D * 2));
+        }
+    }
     // the previous kernel on the stream has completed: inputs may now be read
     wait_previous_kernel();
     allow_next_kernel();
 
-    const int groups = p.H / G;
     // stage list: stage 0 = the chunk's frames, then the ring boxes whose bit is set
     const int n_ring = __popc(p.ring_box_mask);
     const int n_stages = 1 + n_ring;
