@@ -471,7 +471,10 @@ def run_ca2(args):
     share_w = avg_w / step_s
     dom = "temporal" if share_t >= share_s else "spatial"
     dk = kernels[dom]
-    traffic = committed_traffic("k_temporal.cu" if dom == "temporal" else "k_spatial.cu")
+    # the committed capture is of one Open-Sora-shaped launch (B = 1, Pmax = 41, all heads):
+    # other settings' launches move other byte counts
+    captured_shape = args.config == "os_p41" and not sharded
+    traffic = committed_traffic("k_temporal.cu" if dom == "temporal" else "k_spatial.cu") if captured_shape else None
     roofline = {"kernel": "k_temporal_causal" if dom == "temporal" else "k_spatial_prefix",
                 "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
                 "frac": dk["frac"], "traffic": traffic, "peak_source": pk_kind}
