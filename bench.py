@@ -182,6 +182,17 @@ def max_over_ranks(ms: float, dist, world: int, device) -> float:
     return float(tt.item())
 
 
+def job_tokens_per_step(tokens_per_step: int, sharded: bool, world: int, heads: int, heads_all: int) -> float:
+    """Query tokens the whole job moves through attention per step: every replica its own; a
+    head split over `world` ranks moves each token once over all of them; one group of a split
+    timed alone (world 1) counts its heads' share of each token."""
+    if not sharded:
+        return tokens_per_step * world
+    if world > 1:
+        return tokens_per_step
+    return tokens_per_step * heads / heads_all
+
+
 def whole_job_rate(tokens_per_step: int, steps: int, world: int, ms: float) -> float:
     """Query tokens per second of the whole job: every rank's tokens over the slowest rank's time."""
     return tokens_per_step * steps * world / (ms / 1e3)
@@ -371,15 +382,7 @@ def run_ca2(args):
     resident_gb = (cache.tbuf.numel() + cache.sbuf.numel() + NL * 8 * B * l * HW * H_all * D) * 2 / 1e9
     launches_per_step = (T + 1) * NL * 2 + 1
     tokens_per_step = (T + 1) * NL * B * l * HW
-    # query tokens the whole job moves through attention per step: every replica its own; a
-    # head split moves each token once over all ranks, and one group timed alone counts its
-    # heads' share
-    if not sharded:
-        job_tokens = tokens_per_step * world
-    elif world > 1:
-        job_tokens = tokens_per_step
-    else:
-        job_tokens = tokens_per_step * H / H_all
+    job_tokens = job_tokens_per_step(tokens_per_step, sharded, world, H, H_all)
     value = whole_job_rate(job_tokens, args.steps, 1, ms)
 
     # ---- cyclic TPE add (a next-row kernel, timed on its own, outside the step) ----

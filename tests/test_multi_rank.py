@@ -149,3 +149,16 @@ def test_two_ranks_split_heads_and_assemble_the_full_result():
         expect.append((ring.head, ring.count, len(ring.spatial_ids), ring.frames_written))
     assert states[0][0] == expect
     assert sum(s[1] for s in states) == full_bytes[0] and sum(s[2] for s in states) == full_bytes[1]
+
+
+def test_job_tokens_by_parallelism():
+    """Replicas count every rank's tokens; a head split over N ranks counts each token once; one
+    group of a split timed alone counts its heads' share (the groups of a split add up to one)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from causal_kv_cache_b200 import ca2
+    assert bench.job_tokens_per_step(2048, False, 1, 16, 16) == 2048
+    assert bench.job_tokens_per_step(2048, False, 4, 16, 16) == 4 * 2048
+    assert bench.job_tokens_per_step(2048, True, 4, 4, 16) == 2048
+    shares = [bench.job_tokens_per_step(2048, True, 1, ca2.ca2_head_shard(16, 3, r)[1], 16) for r in range(3)]
+    assert sum(shares) == pytest.approx(2048)
