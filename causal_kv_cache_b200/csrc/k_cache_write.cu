@@ -4,10 +4,10 @@
 // one clean forward pass computes its K/V, which join the temporal queue (FIFO, at most
 // Pmax frames) and replace the one-chunk spatial cache.  This kernel is the data movement
 // of that step for every layer at once: a copy, 16 bytes per access (K bit for bit, V as
-// the exact fp16 form of each bf16 value).  The ring
-// is token-major and head-major within a token ([B][HW][H][Pmax][D]: one head's Pmax slots
-// are contiguous), so a temporal write moves each (token, frame, head) row of D elements of
-// the chunk into that head's slot.
+// the exact fp16 form of each bf16 value).  The ring is token-major and head-major within a
+// token ([B][HW][H][Pmax][D]: one head's Pmax slots are contiguous), so a temporal write
+// moves the chunk's n rows of D elements of each (token, head) into n consecutive slots of
+// that head.
 #include <cstdint>
 
 #include "ca2_device.cuh"
