@@ -304,3 +304,37 @@ def test_head_shard_partition():
         with pytest.raises(ca2.Ca2Error) as e:
             ca2.ca2_head_shard(*bad)
         assert e.value.status == -2
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/ca2.h compiles as C99 with warnings as errors, and a C program that calls the
+    library through it links against libca2.so and runs the host-only calls."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_ca2.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "ca2.h"
+int main(void)
+{
+    ca2_config c = {2, 1, 16, 2, 16, 4, 9, 1, 0, 0};
+    size_t tb = 0, sb = 0;
+    int h0 = -1, hc = -1;
+    if (ca2_cache_bytes(&c, &tb, &sb) != CA2_OK) return 1;
+    if (ca2_head_shard(5, 2, 1, &h0, &hc) != CA2_OK || h0 != 3 || hc != 2) return 2;
+    if (ca2_head_shard(1, 2, 0, &h0, &hc) != CA2_ERR_SHAPE) return 3;
+    printf("%zu %zu %s\n", tb, sb, ca2_status_string(CA2_ERR_RANGE));
+    return 0;
+}
+''')
+    exe = tmp_path / "use_ca2"
+    lib_dir = os.path.dirname(ca2.LIBRARY_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe), "-L", lib_dir, "-lca2", "-Wl,-rpath," + lib_dir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    tb, sb = ca2.ca2_cache_bytes(cfg(n_layers=2, hw=16, heads=2, head_dim=16, chunk_len=4, p_max=9, p_spatial=1))
+    assert r.stdout.split()[:2] == [str(tb), str(sb)]
