@@ -26,12 +26,12 @@
  *     void*; NULL = the legacy default stream) and never synchronise.  Ring indices live
  *     on the host and reach the kernels as launch arguments, so host state advances at
  *     call time: issue calls in the order they must execute.
- *   - The attention calls (and ca2_tpe_add) are launched with programmatic dependent
- *     launch: their CTAs may start their set-up while the previous kernel on the stream
- *     drains, but read no input and write no output before it has completed.  Before that
- *     point the temporal call only asks L2 to prefetch ring data of this cache (a hint
- *     with no visible effect), so the caller may write any buffer in the previous kernel.
- *     The cache buffers themselves are written only through this library.
+ *   - The attention calls, ca2_kv_proj_write and ca2_tpe_add are launched with
+ *     programmatic dependent launch: their CTAs may start their set-up while the previous
+ *     kernel on the stream drains, but read no input and write no output before it has
+ *     completed.  Before that point the temporal call only asks L2 to prefetch ring data of
+ *     this cache, a hint with no visible effect (L2 is the point of coherence), so the
+ *     previous kernel may write any buffer, the caches included.
  *   - Errors are returned as ca2_status codes.  Nothing aborts, throws or traps.  A
  *     launch failure is CA2_ERR_CUDA.  A kernel whose bounded wait gave up records it in a
  *     device status word, read (with a device synchronisation) by ca2_device_status.
