@@ -40,6 +40,18 @@ def test_tiny_peaky_values():
         lp.ar_step(wl.chunk_len, 1)
 
 
+def test_tiny_eight_times_scale():
+    """The tiny workload with inputs at 8 times its N(0, 1/16) scale (N(0, 4)): scores of
+    several units, near one-hot softmax rows, running maxima that jump between blocks."""
+    from tests.gpu_util import Loop
+    wl = _wl("tiny", scale=2.0, name="tiny_x8")
+    lp = Loop(wl, seed=9)
+    lp.first_frame()
+    for _ in range(wl.ar_steps):
+        lp.ar_step(wl.chunk_len, wl.denoise_steps)
+    assert len(lp.stats) == 2 * (1 + 3 * 3)
+
+
 def test_first_frame_temporal_returns_v_exactly():
     """Single visible key: with an empty queue and one frame the softmax weight is exactly
     1, so the output is V: bit for bit wherever fp16 (the operand type of the P V product)
