@@ -162,3 +162,23 @@ def test_job_tokens_by_parallelism():
     assert bench.job_tokens_per_step(2048, True, 4, 4, 16) == 2048
     shares = [bench.job_tokens_per_step(2048, True, 1, ca2.ca2_head_shard(16, 3, r)[1], 16) for r in range(3)]
     assert sum(shares) == pytest.approx(2048)
+
+
+def test_reference_arm_line_has_the_contract_keys():
+    """Rank 0 of the reference arm (the oracle on the host cores) prints one JSON line with the
+    keys the bench contract names, its cpu_baseline and e2e describing the same run."""
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
