@@ -90,7 +90,8 @@ typedef enum {
     CA2_ERR_CUDA = -5,      /* a CUDA runtime call or kernel launch failed                */
     CA2_ERR_TIMEOUT = -6,   /* a kernel's bounded wait gave up (see ca2_device_status)     */
     CA2_ERR_RANGE = -7,     /* a device input outside the supported range (see
-                               ca2_device_status): spatial attention takes |V| <= 65504    */
+                               ca2_device_status): V values beyond |v| <= 65504, the fp16
+                               range the caches and the P V products hold V in           */
     CA2_ERR_BOUNDS = -8     /* debug build only: a kernel's bounds check failed and the
                                access was skipped (see ca2_device_status, ca2_debug_build) */
 } ca2_status;
